@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the windowed-attention hot path; prints ONE JSON line (rank 0).
+
+Workload (default): Qwen2.5-0.5B-shaped single-layer prefill, B=1, Hq=14,
+Hkv=2 (GQA), D=64, RoPE base 1e6, N=32768, k=8, bf16 inputs i.i.d. N(0,1)
+from seed 1, plus the decode of the last row against the same K/V.  One step =
+RoPE pre-pass (q and k) -> windowed tcgen05 prefill -> split-KV decode ->
+merge: every row of the hot path.  `value` is prefill tokens/s (B*N tokens
+per step) with inputs resident in HBM; L2 (126 MB) is flushed before every
+step by writing a 256 MiB buffer outside the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 (torchrun): every rank runs an independent replica of the workload on
+its own GPU (the path has no exchange step); time = max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill tokens/s + decode µs/token vs N; % of bf16 TC / HBM roofline"
+WORKLOAD = {
+    "workload": "Qwen2.5-0.5B-shaped single-layer windowed prefill + decode of the last row",
+    "B": 1, "Hq": 14, "Hkv": 2, "D": 64, "N": 32768, "rope_base": 1e6, "k_window": 8.0, "seed": 1,
+}
+L2_FLUSH_BYTES = 256 << 20
+KERNELS_PER_STEP = 5  # rope_pack(q), rope_pack(k), prefill_tc, decode_split, decode_merge
+
+# DRAM bytes per launch of the tcgen05 prefill kernel on this workload, from one
+# ncu capture (profiles/prefill_tc_qwen05b_32k.md).  Valid only while the
+# kernel source hashes to `source_sha1`; otherwise the line reports null.
+TRAFFIC = {"bytes_per_launch": None, "source_sha1": None}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--N", type=int, default=None, help="override sequence length (sweeps)")
+    p.add_argument("--k-window", type=float, default=None, help="override k (inf = window off)")
+    return p.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_sha1():
+    path = os.path.join(ROOT, "long_context_attention_pair_b200", "csrc", "prefill_tc.cu")
+    with open(path, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value, world, device):
+    """Max of a float over ranks (host plumbing only)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.error = None
+
+    def _gpu_id(self):
+        import torch
+        try:
+            u = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:  # noqa: BLE001
+            return str(self.dev)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self._gpu_id(), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception as e:  # noqa: BLE001
+            self.error = str(e)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"error": self.error or "nvidia-smi unavailable"}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:  # noqa: BLE001
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[3:]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"error": "no samples", "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- CPU oracle
+def cpu_baseline(q, k, v, wl, budget_s=12.0):
+    """The fp64 oracle, as it stands, on a bounded sample of query rows (all heads)."""
+    import numpy as np
+    import oracle
+    N = wl["N"]
+    kh = k[0].float().cpu().numpy()
+    vh = v[0].float().cpu().numpy()
+    rng = np.random.default_rng(1234)
+
+    def run(nrows):
+        rows = np.sort(rng.choice(N, size=nrows, replace=False))
+        qh = q[0, rows].float().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.prefill_rows(qh, rows, kh, vh, wl["rope_base"], wl["k_window"])
+        return time.perf_counter() - t0
+
+    t = run(8)
+    nrows = int(max(8, min(1024, 8 * budget_s / max(t, 1e-3))))
+    t = run(nrows)
+    return {"value": nrows / t, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{nrows} uniformly drawn query rows x all {wl['Hq']} heads of the workload "
+                      f"(each row attends its full causal prefix), {t:.1f} s"}
+
+
+def run_reference(args, wl):
+    """Reference arm: the fp64 oracle on the host cores, bounded sample per step."""
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from long_context_attention_pair_b200 import synthetic
+    N, rows_per_step = wl["N"], 4
+    shape_kv = (wl["B"], N, wl["Hkv"], wl["D"])
+    k = synthetic.tensor(wl["seed"], "k", shape_kv, "bf16")[0]
+    v = synthetic.tensor(wl["seed"], "v", shape_kv, "bf16")[0]
+    rng = np.random.default_rng(99)
+    qshape = (wl["B"], N, wl["Hq"], wl["D"])
+
+    def step():
+        rows = np.sort(rng.choice(N, size=rows_per_step, replace=False))
+        qr = synthetic.rows(wl["seed"], "q", qshape, 1, rows, "bf16")[0]
+        oracle.prefill_rows(qr, rows, k, v, wl["rope_base"], wl["k_window"])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    t = time.perf_counter() - t0
+    value = args.steps * rows_per_step / t
+    cb = {"value": value, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+          "sample": f"{rows_per_step} random query rows x all heads per step"}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": dict(wl), "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------------- our arm
+def run_ours(args, wl):
+    import torch
+    import long_context_attention_pair_b200 as atf
+    from long_context_attention_pair_b200 import synthetic
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    B, N, Hq, Hkv, D = wl["B"], wl["N"], wl["Hq"], wl["Hkv"], wl["D"]
+    base, kwin = wl["rope_base"], wl["k_window"]
+    q = synthetic.tensor_torch(wl["seed"], "q", (B, N, Hq, D), "bf16", device=dev)
+    k = synthetic.tensor_torch(wl["seed"], "k", (B, N, Hkv, D), "bf16", device=dev)
+    v = synthetic.tensor_torch(wl["seed"], "v", (B, N, Hkv, D), "bf16", device=dev)
+    out = torch.empty_like(q)
+    qpack = torch.empty((B * Hq, D // 16, N, 16), dtype=torch.bfloat16, device=dev)
+    kpack = torch.empty((B * Hkv, D // 16, N, 16), dtype=torch.bfloat16, device=dev)
+    q_last = q[:, N - 1].contiguous()
+    seqlens = torch.full((B,), N, dtype=torch.int32, device=dev)
+    dws = torch.empty(atf.decode_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device=dev)
+    dec_out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(kw, ev=None):
+        atf.rope_pack(q, base, out=qpack)
+        atf.rope_pack(k, base, out=kpack)
+        if ev is not None:
+            ev[0].record(stream)
+        atf.prefill_packed(qpack, kpack, v, base, kw, out=out)
+        if ev is not None:
+            ev[1].record(stream)
+        atf.decode(q_last, k, v, seqlens, base, kw, kv_layout="NHD", out=dec_out, workspace=dws)
+
+    def timed(kw, steps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for e in evs:
+            flush.zero_()
+            e[0].record(stream)
+            step(kw, (e[1], e[2]))
+            e[3].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        step_ms = [a.elapsed_time(d) for a, _, _, d in evs]
+        kern_ms = [b.elapsed_time(c) for _, b, c, _ in evs]
+        return sum(step_ms), statistics.mean(kern_ms), statistics.median(step_ms)
+
+    for _ in range(args.warmup):
+        step(kwin)
+        step(math.inf)
+    torch.cuda.synchronize()
+    if atf.device_status() != 0:
+        raise RuntimeError("a kernel's bounded wait ran out during warm-up")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    total_ms, kern_ms, med_ms = timed(kwin, args.steps)
+    clocks = sampler.stop()
+    total_ms = reduce_max(total_ms, world, dev)
+    off_total_ms, off_kern_ms, _ = timed(math.inf, max(3, args.steps // 4))
+    off_total_ms = reduce_max(off_total_ms, world, dev)
+    if atf.device_status() != 0:
+        raise RuntimeError("a kernel's bounded wait ran out in the timed region")
+
+    # Decode alone (one token per sequence), same step otherwise.
+    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(50)]
+    for a, b in dec_ev:
+        flush.zero_()
+        a.record(stream)
+        atf.decode(q_last, k, v, seqlens, base, kwin, kv_layout="NHD", out=dec_out, workspace=dws)
+        b.record(stream)
+    torch.cuda.synchronize()
+    dec_us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in dec_ev)
+
+    tokens_per_step = B * N
+    ms_per_step = total_ms / args.steps
+    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    off_ms_per_step = off_total_ms / max(3, args.steps // 4)
+
+    # Roofline of the dominant kernel (tcgen05 prefill): retained FLOPs only.
+    terms = atf.pruned_terms(N, D, base, kwin)
+    flops = B * Hq * (4 * terms["kept"] + D * N * (N + 1))
+    peaks, src = measured_peaks()
+    long_region = total_ms > 2000.0
+    peak = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
+    achieved = flops / (kern_ms / 1e3) / 1e12
+    traffic = TRAFFIC["bytes_per_launch"] if TRAFFIC["source_sha1"] == kernel_sha1() else None
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": "prefill_tc_kernel<64>",
+                "kernel_ms": round(kern_ms, 4),
+                "peak_source": f"{src} ({'sustained' if long_region else 'burst'} bf16)",
+                "flops_per_launch": flops}
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(wl, l2="flushed before every step (256 MiB write, outside the timed events)",
+                       parallelism="replicas" if world > 1 else "single GPU"),
+        "roofline": roofline,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clocks,
+        "window_off": {"ms_per_step": round(off_ms_per_step, 4),
+                       "value": round(world * tokens_per_step / (off_ms_per_step / 1e3), 1),
+                       "prefill_kernel_ms": round(off_kern_ms, 4)},
+        "on_off_speedup": round(off_ms_per_step / ms_per_step, 4),
+        "prefill_kernel_on_off_speedup": round(off_kern_ms / kern_ms, 4),
+        "decode": {"us_per_call": round(dec_us, 2), "us_per_token": round(dec_us / B, 2), "L": N},
+        "pruned_fraction": round(terms["pruned"] / terms["total"], 6),
+        "median_step_ms": round(med_ms, 4),
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = e2e(atf, q, k, v, wl, args, dev, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(q, k, v, wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def e2e(atf, q, k, v, wl, args, dev, world):
+    """Same metric through the public API with host buffers: H2D inputs, prefill,
+    decode of the last row, D2H outputs, all inside the timed region."""
+    import torch
+    B, N, Hq, Hkv, D = wl["B"], wl["N"], wl["Hq"], wl["Hkv"], wl["D"]
+    base, kwin = wl["rope_base"], wl["k_window"]
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hsl = torch.full((B,), N, dtype=torch.int32).pin_memory()
+    hout = torch.empty((B, N, Hq, D), dtype=torch.bfloat16).pin_memory()
+    hdec = torch.empty((B, Hq, D), dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dsl = torch.empty((B,), dtype=torch.int32, device=dev)
+    dout = torch.empty_like(q)
+    ws = torch.empty(atf.prefill_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device=dev)
+    dws = torch.empty(atf.decode_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    steps = max(3, args.steps // 10)
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dsl.copy_(hsl, non_blocking=True)
+        atf.prefill(dq, dk, dv, base, kwin, out=dout, workspace=ws)
+        dec = atf.decode(dq[:, N - 1].contiguous(), dk, dv, dsl, base, kwin, kv_layout="NHD", workspace=dws)
+        hout.copy_(dout, non_blocking=True)
+        hdec.copy_(dec, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = reduce_max(a.elapsed_time(b), world, dev)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsl))
+    d2h = sum(t.numel() * t.element_size() for t in (hout, hdec))
+    return {"value": round(world * B * N * steps / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / steps, 4)}
+
+
+def main():
+    args = parse()
+    if args.steps < 1 or args.warmup < 3:
+        raise SystemExit("need --steps >= 1 and --warmup >= 3")
+    wl = dict(WORKLOAD)
+    if args.N:
+        wl["N"] = args.N
+    if args.k_window is not None:
+        wl["k_window"] = args.k_window
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+/*
+ * atflash.h — C ABI of the B200 (sm_100a) per-RoPE-wavelength windowed
+ * attention library (libatflash.so).
+ *
+ * The method ("ATFlash — Per-RoPE-Wavelength Attention Windows",
+ * gh.bsm-lab.com/ATFlash/ATFlash-Kernel, section "The idea"; arXiv 2608.02947
+ * abstract): in causal attention with rotate-half RoPE, the query-key score is
+ * a sum over D/2 frequency pairs, pair r = dims (r, r + D/2), rotated by
+ * position * theta_r with theta_r = base^(-2r/D).  The term of pair r is kept
+ * only while the distance n - m <= w_r = floor(k * lambda_r), lambda_r =
+ * 2*pi/theta_r; the kept terms feed an unchanged softmax and P.V product.
+ * k = +INFINITY keeps every term (plain causal RoPE attention).  A cell whose
+ * every pair is pruned scores 0 (the empty sum); no key is dropped.
+ *
+ * Conventions shared by every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, unless a
+ *    call says otherwise.  They must stay valid until the work queued on
+ *    `stream` has finished.  The library keeps no reference after returning.
+ *  - GPU calls are asynchronous on `stream` (0 = legacy default stream).
+ *  - Every call validates its arguments first and returns a status < 0 with
+ *    nothing launched when they are invalid.  ATFLASH_OK (0) means the work
+ *    was queued.  Faults inside a queued kernel surface as CUDA errors on the
+ *    stream; a kernel whose bounded internal wait ran out records
+ *    ATFLASH_ERR_TIMEOUT, read back with atflash_device_status().
+ *  - Softmax scale is 1/sqrt(D).  Query head h reads KV head h / (Hq / Hkv).
+ *  - Positions: prefill queries and keys sit at 0..N-1; a decode query of
+ *    sequence b sits at seqlens[b]-1 and attends cache rows 0..seqlens[b]-1.
+ *  - w_r is computed once on the host in fp64 and never in fp32.
+ */
+#ifndef ATFLASH_H
+#define ATFLASH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t. */
+typedef struct CUstream_st *cudaStream_t;
+
+/* Status codes. */
+#define ATFLASH_OK 0
+#define ATFLASH_ERR_INVALID_ARG (-1) /* null pointer, non-positive size, Hq % Hkv != 0, NaN or
+                                        negative k, base <= 1, N beyond 2^31-1 */
+#define ATFLASH_ERR_UNSUPPORTED (-2) /* a head dim or dtype combination with no kernel */
+#define ATFLASH_ERR_WORKSPACE (-3)   /* workspace missing or smaller than required */
+#define ATFLASH_ERR_CUDA (-4)        /* a CUDA runtime/driver call or launch failed */
+#define ATFLASH_ERR_TIMEOUT (-5)     /* a kernel's bounded wait ran out (device status) */
+#define ATFLASH_ERR_ALIGNMENT (-6)   /* a pointer is not 16-byte aligned */
+
+/* Element types of tensors passed to the GPU calls. */
+#define ATFLASH_F32 0
+#define ATFLASH_BF16 1
+
+/* KV-cache layouts accepted by atflash_decode. */
+#define ATFLASH_KV_HND 0 /* [B][Hkv][Nmax][D]: one contiguous block per (sequence, KV head) */
+#define ATFLASH_KV_NHD 1 /* [B][Nmax][Hkv][D]: token-major, the prefill's k/v layout */
+
+/* Text of a status code (static storage, never NULL). */
+const char *atflash_status_string(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int atflash_version(void);
+
+/*
+ * Per-pair window table ("The idea": w_r = k * lambda_r, kept while n - m <= w_r).
+ *   D         head dim, even, 2..256
+ *   rope_base RoPE base (> 1)
+ *   k_window  k >= 0, or +INFINITY for no window
+ *   N         sequence length (>= 1); entries are clamped to N - 1
+ *   w_out     HOST array of D/2 int64 written with min(floor(k*lambda_r), N-1)
+ * Host only; no device work.
+ */
+int atflash_window_table(int D, double rope_base, double k_window, int64_t N, int64_t *w_out);
+
+/* Counts of query-key inner-product terms of ONE (sequence, head) over the
+ * causal triangle of N positions.  A pair-term is one (n, m, r) with m <= n;
+ * a dim-term is one of its two products (so dims = 2 x pairs). */
+typedef struct {
+    uint64_t total;      /* (D/2) * N(N+1)/2 pair-terms */
+    uint64_t kept;       /* pair-terms with n - m <= w_r */
+    uint64_t pruned;     /* total - kept */
+    uint64_t total_dims; /* 2 * total */
+    uint64_t kept_dims;  /* 2 * kept */
+} atflash_terms;
+
+/*
+ * Input-independent closed-form count of kept and pruned terms (arXiv
+ * 2608.02947 abstract: "the reduction rate is input-independent, with a
+ * closed form"; README "The idea": "you know the cost before running").
+ * kept = sum_r (W_r + 1)(2N - W_r)/2 with W_r = min(w_r, N - 1).
+ * Host only; `out` is a HOST pointer.
+ */
+int atflash_pruned_terms(int64_t N, int D, double rope_base, double k_window, atflash_terms *out);
+
+/*
+ * Windowed causal RoPE prefill, bf16 in and out (the spec call).
+ *   q    [B][N][Hq][D]  bf16, un-rotated queries, row-major
+ *   k, v [B][N][Hkv][D] bf16, un-rotated keys, values
+ *   out  [B][N][Hq][D]  bf16, written
+ *   D in {64, 128}; B, Hq, Hkv, N >= 1; Hq % Hkv == 0; N <= 2^31 - 1.
+ * Scratch (rotated Q and K, atflash_prefill_workspace_bytes()) is taken from
+ * a stream-ordered pool owned by the library and returned on `stream`; use
+ * atflash_prefill_ex with a caller workspace to avoid that.
+ * All pointers 16-byte aligned.
+ */
+int atflash_prefill(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
+                    int64_t N, int D, double rope_base, double k_window, cudaStream_t stream);
+
+/* Device scratch bytes atflash_prefill_ex needs (0 on invalid arguments). */
+size_t atflash_prefill_workspace_bytes(int B, int Hq, int Hkv, int64_t N, int D, int in_dtype);
+
+/*
+ * Prefill with explicit dtypes, optional log-sum-exp and a caller workspace.
+ *   in_dtype  ATFLASH_BF16: tensor-core path (tcgen05, bf16 operands, fp32
+ *             accumulate), D in {64, 128}.
+ *             ATFLASH_F32: exact fp32 CUDA-core path, any even D in 2..256.
+ *   out_dtype ATFLASH_BF16 or ATFLASH_F32 (out's element type).
+ *   lse       NULL, or [B][Hq][N] fp32 device array written with the natural
+ *             log-sum-exp of each row's scaled scores.
+ *   workspace device buffer of >= atflash_prefill_workspace_bytes(...) bytes,
+ *             256-byte aligned; owned by the caller, free for reuse once the
+ *             call's work on `stream` has finished.
+ */
+int atflash_prefill_ex(const void *q, const void *k, const void *v, void *out, int B, int Hq,
+                       int Hkv, int64_t N, int D, double rope_base, double k_window, int in_dtype,
+                       int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
+
+/*
+ * RoPE pre-pass on its own: rotate x [B][N][H][D] (positions 0..N-1) once and
+ * write the layout atflash_prefill_packed reads.
+ *   in_dtype ATFLASH_BF16: y is [B*H][D/16][N][16] bf16 ("packed"): chunk c
+ *            holds pairs 8c..8c+7 of each token as (x~_r, x~_{r+D/2})
+ *            interleaved, one 32-byte tensor-core K-step per token; D in {64, 128}.
+ *            ATFLASH_F32: y is [B*H][N][D] fp32, pair-interleaved; even D <= 256.
+ *   y must hold atflash_rope_pack_bytes(B, N, H, D, in_dtype) bytes, 256-byte aligned.
+ * Angles position * theta_r are reduced modulo 2*pi in fp64.
+ */
+int atflash_rope_pack(const void *x, void *y, int B, int64_t N, int H, int D, double rope_base, int in_dtype,
+                      cudaStream_t stream);
+size_t atflash_rope_pack_bytes(int B, int64_t N, int H, int D, int in_dtype);
+
+/*
+ * Windowed attention over already rotated, packed queries and keys (outputs of
+ * atflash_rope_pack with the same in_dtype, B, N, D and rope_base).  Same
+ * semantics, layouts of v/out/lse and constraints as atflash_prefill_ex.
+ */
+int atflash_prefill_packed(const void *qpack, const void *kpack, const void *v, void *out, int B, int Hq,
+                           int Hkv, int64_t N, int D, double rope_base, double k_window, int in_dtype,
+                           int out_dtype, float *lse, cudaStream_t stream);
+
+/* Device scratch bytes atflash_decode needs (0 on invalid arguments). */
+size_t atflash_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D);
+
+/*
+ * Windowed decode: one query token per sequence over a contiguous KV cache
+ * (README "Numbers"/"Using the ports": the window is one more condition on
+ * which K elements are loaded).  Split-KV: each CTA streams one slice of one
+ * sequence's cache, loading only the K dims kept at that slice's distances,
+ * and a second kernel merges the slices' softmax states.
+ *   q              [B][Hq][D]        un-rotated query of each sequence
+ *   kcache, vcache keys (un-rotated unless kcache_rotated) and values, in
+ *                  kv_layout ATFLASH_KV_HND [B][Hkv][Nmax][D] or
+ *                  ATFLASH_KV_NHD [B][Nmax][Hkv][D]
+ *   seqlens        [B] int32 device array, 1 <= seqlens[b] <= Nmax; the query
+ *                  of sequence b sits at position seqlens[b] - 1
+ *   out            [B][Hq][D] written (out_dtype)
+ *   kcache_rotated 0: keys are rotated on load; 1: keys already rotated
+ *   in_dtype       element type of q, kcache, vcache (ATFLASH_BF16 or ATFLASH_F32)
+ *   workspace      device buffer of >= atflash_decode_workspace_bytes(...) bytes
+ *   D in {64, 128}.
+ */
+int atflash_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens,
+                   void *out, int B, int Hq, int Hkv, int64_t Nmax, int D, double rope_base,
+                   double k_window, int kcache_rotated, int kv_layout, int in_dtype, int out_dtype,
+                   void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Device status word of the current device: ATFLASH_OK, or ATFLASH_ERR_TIMEOUT
+ * when a kernel's bounded wait ran out since the last clear.  Synchronises
+ * the device.  clear != 0 resets the word.
+ */
+int atflash_device_status(int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATFLASH_H */

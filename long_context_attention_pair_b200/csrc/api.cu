@@ -1,0 +1,308 @@
+// C ABI of libatflash.so (declared in include/atflash.h): argument checks,
+// the fp64 window table, workspace carving and the kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "internal.h"
+
+namespace atf {
+
+// Device status word: kernels whose bounded wait ran out record it here.
+__device__ int g_device_status;
+
+static std::mutex g_mu;
+static int *g_status_ptr[64];
+static cudaMemPool_t g_pool[64];
+
+static int *status_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<int *>(p);
+    }
+    return g_status_ptr[dev];
+}
+
+// Stream-ordered pool for the scratch of atflash_prefill (kept cached: no
+// release back to the driver between calls).
+static cudaMemPool_t scratch_pool() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_pool[dev]) {
+        cudaMemPoolProps props;
+        memset(&props, 0, sizeof(props));
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+        uint64_t keep = UINT64_MAX;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        g_pool[dev] = pool;
+    }
+    return g_pool[dev];
+}
+
+EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+static uint64_t wait_limit_ns() {
+    static uint64_t v = 0;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char *e = getenv("ATFLASH_WAIT_LIMIT_MS");
+        double ms = e ? atof(e) : 2000.0;
+        if (!(ms > 0)) ms = 2000.0;
+        v = (uint64_t)(ms * 1e6);
+    });
+    return v;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int check_window_args(int D, double base, double k) {
+    if (D < 2 || D > 2 * kMaxPairs || (D & 1) || !(base > 1.0) || isnan(k) || k < 0.0)
+        return ATFLASH_ERR_INVALID_ARG;
+    return ATFLASH_OK;
+}
+
+static int check_shape(int B, int Hq, int Hkv, int64_t N) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || N > INT32_MAX) return ATFLASH_ERR_INVALID_ARG;
+    if ((int64_t)B * Hq > 65535 || (int64_t)B * Hkv * 8 > INT32_MAX) return ATFLASH_ERR_INVALID_ARG;
+    return ATFLASH_OK;
+}
+
+static int fill_window(WindowParams &wp, int D, double base, double k, int64_t N) {
+    int64_t w[kMaxPairs];
+    int rc = window_table(D, base, k, N, w);
+    if (rc != ATFLASH_OK) return rc;
+    memset(&wp, 0, sizeof(wp));
+    wp.H = D / 2;
+    for (int r = 0; r < D / 2; ++r) wp.w[r] = (int32_t)w[r];  // <= N-1 <= INT32_MAX
+    theta_table(D, base, wp.theta);
+    return ATFLASH_OK;
+}
+
+static size_t prefill_ws(int B, int Hq, int Hkv, int64_t N, int D, int in_dtype) {
+    const size_t es = (in_dtype == ATFLASH_F32) ? 4 : 2;
+    return align256((size_t)B * Hq * N * D * es) + align256((size_t)B * Hkv * N * D * es);
+}
+
+}  // namespace atf
+
+using namespace atf;
+
+extern "C" {
+
+const char *atflash_status_string(int status) {
+    switch (status) {
+        case ATFLASH_OK: return "ok";
+        case ATFLASH_ERR_INVALID_ARG: return "invalid argument";
+        case ATFLASH_ERR_UNSUPPORTED: return "unsupported head dim or dtype";
+        case ATFLASH_ERR_WORKSPACE: return "workspace missing or too small";
+        case ATFLASH_ERR_CUDA: return "CUDA runtime or launch error";
+        case ATFLASH_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
+        case ATFLASH_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        default: return "unknown status";
+    }
+}
+
+int atflash_version(void) { return 100; }
+
+int atflash_window_table(int D, double rope_base, double k_window, int64_t N, int64_t *w_out) {
+    if (!w_out) return ATFLASH_ERR_INVALID_ARG;
+    return window_table(D, rope_base, k_window, N, w_out);
+}
+
+int atflash_pruned_terms(int64_t N, int D, double rope_base, double k_window, atflash_terms *out) {
+    return pruned_terms(N, D, rope_base, k_window, out);
+}
+
+size_t atflash_prefill_workspace_bytes(int B, int Hq, int Hkv, int64_t N, int D, int in_dtype) {
+    if (check_shape(B, Hq, Hkv, N) != ATFLASH_OK || D < 2 || D > 2 * kMaxPairs || (D & 1)) return 0;
+    if (in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) return 0;
+    return prefill_ws(B, Hq, Hkv, N, D, in_dtype);
+}
+
+static int check_prefill_common(int B, int Hq, int Hkv, int64_t N, int D, double base, double k, int in_dtype,
+                                int out_dtype) {
+    int rc = check_shape(B, Hq, Hkv, N);
+    if (rc != ATFLASH_OK) return rc;
+    if ((rc = check_window_args(D, base, k)) != ATFLASH_OK) return rc;
+    if ((in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) ||
+        (out_dtype != ATFLASH_F32 && out_dtype != ATFLASH_BF16))
+        return ATFLASH_ERR_UNSUPPORTED;
+    if (in_dtype == ATFLASH_BF16 && D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
+    return ATFLASH_OK;
+}
+
+static int run_prefill_packed(const void *qt, const void *kt, const void *v, void *out, int B, int Hq, int Hkv,
+                              int64_t N, int D, double base, double k, int in_dtype, int out_dtype, float *lse,
+                              cudaStream_t stream) {
+    WindowParams wp;
+    int rc = fill_window(wp, D, base, k, N);
+    if (rc != ATFLASH_OK) return rc;
+    Problem p{B, Hq, Hkv, D, N};
+    const int out_f32 = (out_dtype == ATFLASH_F32);
+    cudaError_t e;
+    if (in_dtype == ATFLASH_BF16) {
+        int *status = status_word();
+        if (!status) return ATFLASH_ERR_CUDA;
+        e = launch_prefill_tc(qt, kt, v, out, out_f32, lse, p, wp, status, wait_limit_ns(), stream);
+    } else {
+        e = launch_prefill_simt_f32((const float *)qt, (const float *)kt, (const float *)v, out, out_f32, lse, p,
+                                    wp, stream);
+    }
+    return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
+}
+
+static int run_rope_pack(const void *x, void *y, int B, int64_t N, int H, int D, double base, int in_dtype,
+                         cudaStream_t stream) {
+    WindowParams wp;
+    memset(&wp, 0, sizeof(wp));
+    wp.H = D / 2;
+    theta_table(D, base, wp.theta);
+    cudaError_t e = (in_dtype == ATFLASH_BF16) ? launch_rope_pack_bf16(x, y, B, N, H, D, wp, stream)
+                                               : launch_rope_pack_f32(x, y, B, N, H, D, wp, stream);
+    return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
+}
+
+size_t atflash_rope_pack_bytes(int B, int64_t N, int H, int D, int in_dtype) {
+    if (check_shape(B, H, H, N) != ATFLASH_OK || D < 2 || D > 2 * kMaxPairs || (D & 1)) return 0;
+    if (in_dtype == ATFLASH_BF16) return (D == 64 || D == 128) ? (size_t)B * H * N * D * 2 : 0;
+    if (in_dtype == ATFLASH_F32) return (size_t)B * H * N * D * 4;
+    return 0;
+}
+
+int atflash_rope_pack(const void *x, void *y, int B, int64_t N, int H, int D, double rope_base, int in_dtype,
+                      cudaStream_t stream) {
+    if (!x || !y) return ATFLASH_ERR_INVALID_ARG;
+    int rc = check_shape(B, H, H, N);
+    if (rc != ATFLASH_OK) return rc;
+    if ((rc = check_window_args(D, rope_base, 0.0)) != ATFLASH_OK) return rc;
+    if (in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) return ATFLASH_ERR_UNSUPPORTED;
+    if (in_dtype == ATFLASH_BF16 && D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
+    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(y) & 255u)) return ATFLASH_ERR_ALIGNMENT;
+    return run_rope_pack(x, y, B, N, H, D, rope_base, in_dtype, stream);
+}
+
+int atflash_prefill_packed(const void *qpack, const void *kpack, const void *v, void *out, int B, int Hq,
+                           int Hkv, int64_t N, int D, double rope_base, double k_window, int in_dtype,
+                           int out_dtype, float *lse, cudaStream_t stream) {
+    if (!qpack || !kpack || !v || !out) return ATFLASH_ERR_INVALID_ARG;
+    int rc = check_prefill_common(B, Hq, Hkv, N, D, rope_base, k_window, in_dtype, out_dtype);
+    if (rc != ATFLASH_OK) return rc;
+    if ((reinterpret_cast<uintptr_t>(qpack) & 255u) || (reinterpret_cast<uintptr_t>(kpack) & 255u) ||
+        !aligned16(v) || !aligned16(out))
+        return ATFLASH_ERR_ALIGNMENT;
+    return run_prefill_packed(qpack, kpack, v, out, B, Hq, Hkv, N, D, rope_base, k_window, in_dtype, out_dtype,
+                              lse, stream);
+}
+
+int atflash_prefill_ex(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
+                       int64_t N, int D, double rope_base, double k_window, int in_dtype, int out_dtype,
+                       float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (!q || !k || !v || !out) return ATFLASH_ERR_INVALID_ARG;
+    int rc = check_prefill_common(B, Hq, Hkv, N, D, rope_base, k_window, in_dtype, out_dtype);
+    if (rc != ATFLASH_OK) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATFLASH_ERR_ALIGNMENT;
+    const size_t need = prefill_ws(B, Hq, Hkv, N, D, in_dtype);
+    if (!workspace || workspace_bytes < need) return ATFLASH_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATFLASH_ERR_ALIGNMENT;
+    const size_t es = (in_dtype == ATFLASH_F32) ? 4 : 2;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *qt = ws;
+    void *kt = ws + align256((size_t)B * Hq * N * D * es);
+    if ((rc = run_rope_pack(q, qt, B, N, Hq, D, rope_base, in_dtype, stream)) != ATFLASH_OK) return rc;
+    if ((rc = run_rope_pack(k, kt, B, N, Hkv, D, rope_base, in_dtype, stream)) != ATFLASH_OK) return rc;
+    return run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, rope_base, k_window, in_dtype, out_dtype, lse,
+                              stream);
+}
+
+int atflash_prefill(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv, int64_t N,
+                    int D, double rope_base, double k_window, cudaStream_t stream) {
+    if (!q || !k || !v || !out) return ATFLASH_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, N);
+    if (rc != ATFLASH_OK) return rc;
+    if ((rc = check_window_args(D, rope_base, k_window)) != ATFLASH_OK) return rc;
+    if (D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
+    const size_t need = prefill_ws(B, Hq, Hkv, N, D, ATFLASH_BF16);
+    cudaMemPool_t pool = scratch_pool();
+    if (!pool) return ATFLASH_ERR_CUDA;
+    void *ws = nullptr;
+    if (cudaMallocFromPoolAsync(&ws, need, pool, stream) != cudaSuccess) return ATFLASH_ERR_CUDA;
+    rc = atflash_prefill_ex(q, k, v, out, B, Hq, Hkv, N, D, rope_base, k_window, ATFLASH_BF16, ATFLASH_BF16,
+                            nullptr, ws, need, stream);
+    cudaFreeAsync(ws, stream);
+    return rc;
+}
+
+size_t atflash_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D) {
+    if (check_shape(B, Hq, Hkv, Nmax) != ATFLASH_OK || (D != 64 && D != 128)) return 0;
+    return decode_workspace_bytes(B, Hq, Nmax, D);
+}
+
+int atflash_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out,
+                   int B, int Hq, int Hkv, int64_t Nmax, int D, double rope_base, double k_window,
+                   int kcache_rotated, int kv_layout, int in_dtype, int out_dtype, void *workspace,
+                   size_t workspace_bytes, cudaStream_t stream) {
+    if (!q || !kcache || !vcache || !seqlens || !out) return ATFLASH_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, Nmax);
+    if (rc != ATFLASH_OK) return rc;
+    if ((rc = check_window_args(D, rope_base, k_window)) != ATFLASH_OK) return rc;
+    if (kcache_rotated != 0 && kcache_rotated != 1) return ATFLASH_ERR_INVALID_ARG;
+    if (kv_layout != ATFLASH_KV_HND && kv_layout != ATFLASH_KV_NHD) return ATFLASH_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
+    if ((in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) ||
+        (out_dtype != ATFLASH_F32 && out_dtype != ATFLASH_BF16))
+        return ATFLASH_ERR_UNSUPPORTED;
+    if (Hq / Hkv > 16) return ATFLASH_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out))
+        return ATFLASH_ERR_ALIGNMENT;
+    const size_t need = decode_workspace_bytes(B, Hq, Nmax, D);
+    if (!workspace || workspace_bytes < need) return ATFLASH_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return ATFLASH_ERR_ALIGNMENT;
+    WindowParams wp;
+    if ((rc = fill_window(wp, D, rope_base, k_window, Nmax)) != ATFLASH_OK) return rc;
+    Problem p{B, Hq, Hkv, D, Nmax};
+    cudaError_t e = launch_decode(q, kcache, vcache, seqlens, out, out_dtype == ATFLASH_F32,
+                                  in_dtype == ATFLASH_F32, kcache_rotated, kv_layout == ATFLASH_KV_NHD, p, wp,
+                                  static_cast<float *>(workspace), stream);
+    return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
+}
+
+int atflash_device_status(int clear) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return ATFLASH_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return ATFLASH_ERR_CUDA;
+    if (clear) {
+        int z = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(int)) != cudaSuccess) return ATFLASH_ERR_CUDA;
+    }
+    return v >= ATFLASH_DEVICE_TIMEOUT_BASE ? ATFLASH_ERR_TIMEOUT : ATFLASH_OK;
+}
+
+}  // extern "C"

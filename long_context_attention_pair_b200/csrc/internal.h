@@ -1,0 +1,62 @@
+// Internal interfaces between the C ABI (api.cu) and the kernel launchers.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "status.h"
+
+namespace atf {
+
+constexpr int kMaxPairs = 128;  // D <= 256
+
+// Host-side window math (window.cpp).  theta_r = base^(-2r/D),
+// lambda_r = 2*pi/theta_r, w_r = floor(k*lambda_r) clamped to N-1.
+int window_table(int D, double base, double k, int64_t N, int64_t *w);
+int pruned_terms(int64_t N, int D, double base, double k, atflash_terms *out);
+void theta_table(int D, double base, double *theta);
+
+// Per-call constants shared by every kernel of one call.
+struct WindowParams {
+    int H;                      // D/2 pairs
+    int32_t w[kMaxPairs];       // per-pair window, clamped to N-1 (non-decreasing in r)
+    double theta[kMaxPairs];    // theta_r in fp64 (RoPE angles are reduced in fp64)
+};
+
+struct Problem {
+    int B, Hq, Hkv, D;
+    int64_t N;
+};
+
+// RoPE pre-pass: rotate q and k once per token into the layouts the prefill
+// kernels read.  bf16 path: packed [b*H+h][D/16][N][16] bf16, pair-interleaved
+// (element 2j of chunk c is x~_{8c+j}, element 2j+1 is x~_{8c+j+D/2}).
+// fp32 path: [b*H+h][N][D] fp32 pair-interleaved.
+cudaError_t launch_rope_pack_bf16(const void *x, void *y, int B, int64_t N, int Hx, int D,
+                                  const WindowParams &wp, cudaStream_t s);
+cudaError_t launch_rope_pack_f32(const void *x, void *y, int B, int64_t N, int Hx, int D,
+                                 const WindowParams &wp, cudaStream_t s);
+
+// Exact fp32 CUDA-core prefill over pre-rotated fp32 Q~/K~.
+cudaError_t launch_prefill_simt_f32(const float *qt, const float *kt, const float *v, void *out, int out_f32,
+                                    float *lse, const Problem &p, const WindowParams &wp, cudaStream_t s);
+
+// tcgen05 prefill over the packed bf16 Q~/K~ and the caller's bf16 V.
+cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *v, void *out, int out_f32,
+                              float *lse, const Problem &p, const WindowParams &wp, int *status,
+                              uint64_t wait_limit_ns, cudaStream_t s);
+
+// Split-KV decode + merge.
+int decode_num_splits(int64_t Nmax);
+size_t decode_workspace_bytes(int B, int Hq, int64_t Nmax, int D);
+cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const int32_t *seqlens, void *out,
+                          int out_f32, int in_f32, int krot, int nhd, const Problem &p,
+                          const WindowParams &wp, float *workspace, cudaStream_t s);
+
+// Driver entry point for cuTensorMapEncodeTiled (resolved once, no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+}  // namespace atf

@@ -100,3 +100,45 @@ def rows(seed: int, name: str, shape, row_axis: int, row_ids, dtype: str = "bf16
     strides = np.cumprod((1,) + shape[::-1][:-1])[::-1]
     flat = sum(g.astype(np.uint64) * np.uint64(st) for g, st in zip(grids, strides))
     return _round(normal_at(seed, STREAMS[name], flat.ravel()), dtype).reshape(flat.shape)
+
+
+# ---------------------------------------------------------------- device twin
+def _i64(u: int) -> int:
+    """uint64 constant as the int64 with the same bits."""
+    return u - (1 << 64) if u >= (1 << 63) else u
+
+
+def _lsr(z, k: int):
+    """Logical right shift of int64 tensors holding uint64 bits."""
+    return (z >> k) & ((1 << (64 - k)) - 1)
+
+
+def _mix_t(z):
+    z = (z ^ _lsr(z, 30)) * _i64(0xBF58476D1CE4E5B9)
+    z = (z ^ _lsr(z, 27)) * _i64(0x94D049BB133111EB)
+    return z ^ _lsr(z, 31)
+
+
+def tensor_torch(seed: int, name: str, shape, dtype: str = "bf16", device="cuda", chunk: int = 1 << 26):
+    """Same draws as ``tensor`` generated with torch ops on ``device`` (int64
+    arithmetic wraps like uint64); returns a torch tensor of dtype bf16/f32."""
+    import torch
+    n = int(np.prod(shape))
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    out = torch.empty(n, dtype=tdt, device=device)
+    key = _i64(int(_key(seed, STREAMS[name])))
+    golden = _i64(int(_GOLDEN))
+    scale = 1.0 / 9007199254740992.0
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        idx = torch.arange(s, e, dtype=torch.int64, device=device)
+        pair = idx >> 1
+        u1 = _lsr(_mix_t(key + (2 * pair + 1) * golden), 11).to(torch.float64)
+        u2 = _lsr(_mix_t(key + (2 * pair + 2) * golden), 11).to(torch.float64)
+        u1 = (u1 + 1.0) * scale
+        u2 = u2 * scale
+        rad = torch.sqrt(-2.0 * torch.log(u1))
+        ang = (2.0 * np.pi) * u2
+        val = torch.where((idx & 1).bool(), rad * torch.sin(ang), rad * torch.cos(ang))
+        out[s:e] = val.to(torch.float32).to(tdt)
+    return out.reshape(tuple(shape))

@@ -1,0 +1,156 @@
+"""Host-side checks of the C ABI (no GPU needed, no compute launched).
+
+* libatflash.so loads and exports every function declared in include/atflash.h;
+* the window table and the closed-form term counts equal the oracle's,
+  bit-exactly, on every workload shape and on edge cases;
+* invalid arguments return the documented status before anything is launched.
+"""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import long_context_attention_pair_b200 as atf
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "atflash.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from long_context_attention_pair_b200 import build
+    build.build()
+    return atf.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(atflash_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_three_north_star_calls():
+    names = declared_functions()
+    for f in ("atflash_prefill", "atflash_decode", "atflash_pruned_terms"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for s in (0, -1, -2, -3, -4, -5, -6):
+        assert atf.status_string(s) != "unknown status"
+
+
+WINDOW_CASES = [
+    (64, 1e4, 1.0, 256), (64, 1e4, math.inf, 256), (64, 1e6, 8.0, 32768), (128, 5e5, 16.0, 131072),
+    (128, 1e7, 16.0, 524288), (128, 1e7, 64.0, 1048576), (128, 1e7, 4.0, 1048576), (8, 10.0, 0.25, 300),
+    (2, 1e4, 0.0, 10), (256, 1e4, 2.5, 5000),
+]
+
+
+@pytest.mark.parametrize("D,base,k,N", WINDOW_CASES)
+def test_window_table_equals_oracle(L, oracle, D, base, k, N):
+    got = np.array(atf.window_table(D, base, k, N), dtype=np.float64)
+    ref = np.minimum(oracle.window_limits(D, base, k), N - 1)
+    np.testing.assert_array_equal(got, ref)
+
+
+@pytest.mark.parametrize("D,base,k,N", WINDOW_CASES + [(64, 1e4, 1.0, 1), (128, 1e7, 16.0, 1 << 26)])
+def test_pruned_terms_equal_oracle_closed_form(L, oracle, D, base, k, N):
+    t = atf.pruned_terms(N, D, base, k)
+    kept, total = oracle.count_closed(N, D, base, k)
+    assert (t["kept"], t["total"]) == (kept, total)
+    assert t["pruned"] == total - kept
+    assert t["kept_dims"] == 2 * kept and t["total_dims"] == 2 * total
+
+
+@pytest.mark.parametrize("N,D,base,k", [(256, 64, 1e4, 1.0), (300, 8, 10.0, 0.25), (513, 128, 5e5, 16.0),
+                                        (1000, 128, 1e7, 4.0)])
+def test_pruned_terms_equal_bruteforce(L, oracle, N, D, base, k):
+    t = atf.pruned_terms(N, D, base, k)
+    assert (t["kept"], t["total"]) == oracle.count_bruteforce(N, D, base, k)
+
+
+def test_pruned_terms_rejects_bad_args(L):
+    t = atf.Terms()
+    for args in [(0, 64, 1e4, 1.0), (256, 63, 1e4, 1.0), (256, 64, 1.0, 1.0), (256, 64, 1e4, -1.0),
+                 (256, 64, 1e4, float("nan")), (256, 512, 1e4, 1.0)]:
+        assert L.atflash_pruned_terms(*args, ctypes.byref(t)) == -1
+    assert L.atflash_pruned_terms(256, 64, 1e4, 1.0, None) == -1
+
+
+# Fake, aligned, never-dereferenced device addresses: every case below must be
+# rejected by the argument checks before any CUDA call.
+P = ctypes.c_void_p(1 << 20)
+
+
+def prefill_ex(L, **kw):
+    a = dict(q=P, k=P, v=P, out=P, B=1, Hq=2, Hkv=1, N=256, D=64, base=1e4, kwin=1.0, ind=atf.BF16,
+             outd=atf.BF16, lse=None, ws=P, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return L.atflash_prefill_ex(a["q"], a["k"], a["v"], a["out"], a["B"], a["Hq"], a["Hkv"], a["N"], a["D"],
+                                a["base"], a["kwin"], a["ind"], a["outd"], a["lse"], a["ws"], a["wsb"],
+                                a["stream"])
+
+
+def test_prefill_argument_errors(L):
+    assert prefill_ex(L, q=None) == -1
+    assert prefill_ex(L, B=0) == -1
+    assert prefill_ex(L, Hq=3, Hkv=2) == -1
+    assert prefill_ex(L, N=0) == -1
+    assert prefill_ex(L, N=1 << 31) == -1
+    assert prefill_ex(L, kwin=-1.0) == -1
+    assert prefill_ex(L, kwin=float("nan")) == -1
+    assert prefill_ex(L, base=1.0) == -1
+    assert prefill_ex(L, D=96) == -2          # no tensor-core kernel for D=96
+    assert prefill_ex(L, ind=7) == -2
+    assert prefill_ex(L, q=ctypes.c_void_p((1 << 20) + 8)) == -6
+    assert prefill_ex(L, ws=None) == -3
+    assert prefill_ex(L, wsb=10) == -3
+    assert prefill_ex(L, ws=ctypes.c_void_p((1 << 20) + 16)) == -6
+
+
+def test_rope_pack_and_packed_prefill_argument_errors(L):
+    assert L.atflash_rope_pack(None, P, 1, 256, 2, 64, 1e4, atf.BF16, None) == -1
+    assert L.atflash_rope_pack(P, P, 1, 256, 2, 96, 1e4, atf.BF16, None) == -2
+    assert L.atflash_rope_pack(P, ctypes.c_void_p((1 << 20) + 32), 1, 256, 2, 64, 1e4, atf.BF16, None) == -6
+    assert L.atflash_rope_pack_bytes(1, 256, 2, 64, atf.BF16) == 256 * 2 * 64 * 2
+    assert L.atflash_rope_pack_bytes(1, 256, 2, 6, atf.F32) == 256 * 2 * 6 * 4
+    assert L.atflash_prefill_packed(P, P, P, None, 1, 2, 1, 256, 64, 1e4, 1.0, atf.BF16, atf.BF16, None,
+                                    None) == -1
+    assert L.atflash_prefill_packed(P, P, P, P, 1, 2, 1, 256, 128, 1e4, -2.0, atf.BF16, atf.BF16, None,
+                                    None) == -1
+
+
+def test_workspace_sizes(L):
+    assert atf.prefill_workspace_bytes(1, 14, 2, 32768, 64) == 14 * 32768 * 64 * 2 + 2 * 32768 * 64 * 2
+    assert atf.prefill_workspace_bytes(1, 1, 1, 256, 64, atf.F32) == 2 * 256 * 64 * 4
+    assert atf.prefill_workspace_bytes(0, 1, 1, 256, 64) == 0
+    assert atf.decode_workspace_bytes(4, 28, 4, 1 << 20, 128) > 0
+    assert atf.decode_workspace_bytes(4, 28, 4, 1 << 20, 96) == 0
+
+
+def test_decode_argument_errors(L):
+    def dec(**kw):
+        a = dict(q=P, kc=P, vc=P, sl=P, out=P, B=4, Hq=28, Hkv=4, Nmax=4096, D=128, base=1e7, kwin=16.0, krot=0,
+                 lay=atf.KV_HND, ind=atf.BF16, outd=atf.F32, ws=P, wsb=1 << 40, stream=None)
+        a.update(kw)
+        return L.atflash_decode(a["q"], a["kc"], a["vc"], a["sl"], a["out"], a["B"], a["Hq"], a["Hkv"],
+                                a["Nmax"], a["D"], a["base"], a["kwin"], a["krot"], a["lay"], a["ind"], a["outd"],
+                                a["ws"], a["wsb"], a["stream"])
+    assert dec(sl=None) == -1
+    assert dec(Hq=30) == -1
+    assert dec(krot=2) == -1
+    assert dec(lay=5) == -1
+    assert dec(D=80) == -2
+    assert dec(Hq=68, Hkv=4) == -2   # more than 16 query heads per KV head
+    assert dec(ws=None) == -3
+    assert dec(wsb=100) == -3
+    assert dec(vc=ctypes.c_void_p((1 << 20) + 4)) == -6
