@@ -89,6 +89,12 @@ def reduce_max(value, world, device):
     return float(t.item())
 
 
+def throughput(world, tokens_per_step, steps, total_ms_max):
+    """Whole-job tokens/s: every rank processed `steps` steps of `tokens_per_step`
+    tokens; the job took the slowest rank's time."""
+    return world * tokens_per_step * steps / (total_ms_max / 1e3)
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -307,7 +313,7 @@ def run_ours(args, wl):
 
     tokens_per_step = B * N
     ms_per_step = total_ms / args.steps
-    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    value = throughput(world, tokens_per_step, args.steps, total_ms)
     off_ms_per_step = off_total_ms / max(3, args.steps // 4)
 
     # Roofline of the dominant kernel (tcgen05 prefill): retained FLOPs only.
