@@ -14,19 +14,27 @@
 // the caller's [B][N][Hkv][D] bf16.  One K-step of the MMA (16 bf16) is one
 // chunk = 8 complete pairs, so the dense contraction over pairs >= 8*floor(r_lo/8)
 // is a run of whole K-steps; the < 8 fully-pruned pairs at the start of the
-// first loaded chunk are zeroed in shared memory before the MMA reads it, and
-// the boundary pairs are subtracted per cell where n - m > w_r.
+// first loaded chunk are zeroed in shared memory before the MMA reads them,
+// and the boundary pairs are subtracted per cell where n - m > w_r.
 //
-// CTA = one (batch*query head, 128-row query tile); 6 warps:
-//   warp 0      TMA producer (Q~ once; K~ chunks and V per key tile, 2 stages)
-//   warp 1      TMEM owner and MMA issuer (S = Q~ K~^T into one of two TMEM
-//               S buffers, O += P V into TMEM O); zeroes pruned pairs
-//   warps 2..5  softmax: one TMEM lane quarter (32 query rows) each; fix-up,
-//               causal mask, online softmax in the log2 domain, O rescale,
-//               P (bf16) to shared memory; epilogue O / l.
+// CTA = one 128-row query tile of TWO query heads of the same GQA group: both
+// heads read the same K/V tiles at the same distances, so they share every
+// load, every pruned-chunk decision and every boundary pair, while their two
+// softmax warpgroups ping-pong with the tensor core.  12 warps:
+//   warps 0-3 / 4-7  softmax of head 0 / head 1: one TMEM lane quarter each;
+//                    boundary fix-up, causal mask, online softmax in the log2
+//                    domain, P (bf16) written back over S in TMEM, O rescale
+//                    (only when the running max grows by more than 2^8),
+//                    epilogue O / l
+//   warp 8           TMA producer (Q~ once; K~ chunks and V per key tile)
+//   warp 9           TMEM owner and MMA issuer: S_h = Q~_h K~^T (smem x smem),
+//                    O_h += P_h V (P from TMEM, V from smem)
+//   warp 10          zeroes the fully-pruned pairs of the first loaded K~ chunk
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D);
+// P_h occupies the first 64 columns of S_h once S_h has been read.
 // Every mbarrier wait is bounded in time; on expiry the CTA records
-// ATFLASH_ERR_TIMEOUT in the device status word, drains its tensor-core work
-// and in-flight copies, frees TMEM and exits.
+// ATFLASH_ERR_TIMEOUT in the device status word, lets its copies land, drains
+// its tensor-core work, frees TMEM and exits.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -39,35 +47,36 @@ namespace tc {
 
 constexpr int kBM = 128;
 constexpr int kBN = 128;
-constexpr int kStages = 2;
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
+constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpFix = 10;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kChunkBytes = kBN * 32;  // 128 rows x 16 bf16 (one K-step)
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
 
 template <int D>
-struct Layout {
-    static constexpr int C = D / 16;                  // chunks (K-steps) of the QK contraction
-    static constexpr int QBytes = C * kChunkBytes;
+struct Cfg {
+    static constexpr int C = D / 16;                  // K-steps of the QK contraction
+    static constexpr int KS = (D == 64) ? 3 : 2;      // K~ stages
+    static constexpr int VS = (D == 64) ? 3 : 2;      // V stages
+    static constexpr int QBytes = C * kChunkBytes;    // one query tile
     static constexpr int KBytes = C * kChunkBytes;
     static constexpr int VBytes = (D / 64) * 16384;   // 128 keys x 64 dims x 2 B per group
-    static constexpr int PBytes = 2 * 16384;          // 128 rows x 128 keys bf16, two 64-key groups
-    static constexpr int OffQ = 0;
-    static constexpr int OffK = OffQ + QBytes;
-    static constexpr int OffV = OffK + kStages * KBytes;
-    static constexpr int OffP = OffV + kStages * VBytes;
-    static constexpr int OffCtl = OffP + PBytes;
-    static constexpr int CtlBytes = 2048;
-    static constexpr int Total = OffCtl + CtlBytes;
-    // At least ~114 KB so that one CTA (and its 512 TMEM columns) owns an SM.
-    static constexpr int Request = (Total + 1024 > 120 * 1024) ? Total + 1024 : 120 * 1024;
+    static constexpr int OffQ = 0;                    // two query tiles
+    static constexpr int OffK = OffQ + 2 * QBytes;
+    static constexpr int OffV = OffK + KS * KBytes;
+    static constexpr int OffCtl = OffV + VS * VBytes;
+    static constexpr int Total = OffCtl + 2048;
+    static constexpr int Request = Total + 1024;
+    static constexpr uint32_t TmemO0 = 256, TmemO1 = 256 + D;
 };
 
+template <int KS, int VS>
 struct Ctl {
     uint64_t q_full;
-    uint64_t k_full[kStages], k_empty[kStages];
-    uint64_t v_full[kStages], v_empty[kStages];
-    uint64_t s_full[2], s_free[2];
-    uint64_t p_full, o_ready, drain;
+    uint64_t k_full[KS], k_ready[KS], k_empty[KS];
+    uint64_t v_full[VS], v_empty[VS];
+    uint64_t s_full[2], p_full[2], o_done[2];
+    uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
     int w[kMaxPairs];
@@ -115,45 +124,54 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ WindowParams wp,
                       void *out, int out_f32, float *lse, int64_t N, int Hq, int Hkv, int *status,
                       uint64_t limit_ns) {
-    using L = Layout<D>;
-    constexpr int C = L::C;
+    using F = Cfg<D>;
+    constexpr int C = F::C;
     constexpr int H = D / 2;
+    constexpr int KS = F::KS, VS = F::VS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sQ = smem + L::OffQ;
-    uint8_t *sK = smem + L::OffK;
-    uint8_t *sV = smem + L::OffV;
-    uint8_t *sP = smem + L::OffP;
-    Ctl *ctl = reinterpret_cast<Ctl *>(smem + L::OffCtl);
+    uint8_t *sQ = smem + F::OffQ;
+    uint8_t *sK = smem + F::OffK;
+    uint8_t *sV = smem + F::OffV;
+    Ctl<KS, VS> *ctl = reinterpret_cast<Ctl<KS, VS> *>(smem + F::OffCtl);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_qt = (int)((N + kBM - 1) / kBM);
     const int qt = num_qt - 1 - (int)blockIdx.x;  // longest query tiles first
-    const int bh = blockIdx.y;
-    const int b = bh / Hq, hq = bh % Hq, kvh = hq / (Hq / Hkv);
+    const int G = Hq / Hkv;
+    const int pairs_per_group = (G + 1) / 2;
+    const int b = blockIdx.y / (Hkv * pairs_per_group);
+    const int rem = blockIdx.y % (Hkv * pairs_per_group);
+    const int kvh = rem / pairs_per_group;
+    const int hp = rem % pairs_per_group;
+    const int h0 = kvh * G + 2 * hp;
+    const bool two = (2 * hp + 1) < G;  // a second head of the group shares this CTA
+    const int nwg = two ? 2 : 1;
     const int64_t n0 = (int64_t)qt * kBM;
     const int nkt = qt + 1;  // key tiles 0..qt (causal)
 
     if (threadIdx.x == 0) {
         mbar_init(&ctl->q_full, 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < KS; ++s) {
             mbar_init(&ctl->k_full[s], 1);
-            mbar_init(&ctl->k_empty[s], 1 + 4);
+            mbar_init(&ctl->k_ready[s], 1);
+            mbar_init(&ctl->k_empty[s], 1 + 4 * nwg);
+        }
+        for (int s = 0; s < VS; ++s) {
             mbar_init(&ctl->v_full[s], 1);
             mbar_init(&ctl->v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&ctl->s_full[s], 1);
-            mbar_init(&ctl->s_free[s], 4);
+            mbar_init(&ctl->p_full[s], 4);
+            mbar_init(&ctl->o_done[s], 1);
         }
-        mbar_init(&ctl->p_full, 4);
-        mbar_init(&ctl->o_ready, 1);
         mbar_init(&ctl->drain, 1);
         ctl->abort_flag = 0;
         fence_mbar_init();
     }
     for (int r = threadIdx.x; r < H; r += kThreads) ctl->w[r] = wp.w[r];
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tmem_alloc(&ctl->tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -164,264 +182,325 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int *w = ctl->w;
     WaitCtl wc{&ctl->abort_flag, status, limit_ns, 0};
 
-    if (warp == 0) {
+    if (warp == kWarpProducer) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            int last_k[kStages] = {-1, -1}, last_v[kStages] = {-1, -1};
-            mbar_expect_tx(&ctl->q_full, L::QBytes);
-            for (int c = 0; c < C; ++c)
-                tma_load_3d(sQ + c * kChunkBytes, &tm_q, &ctl->q_full, 0, (int)n0, bh * C + c);
+            int last_k[KS], last_v[VS];
+            for (int s = 0; s < KS; ++s) last_k[s] = -1;
+            for (int s = 0; s < VS; ++s) last_v[s] = -1;
+            mbar_expect_tx(&ctl->q_full, (uint32_t)(nwg * F::QBytes));
+            for (int t = 0; t < nwg; ++t)
+                for (int c = 0; c < C; ++c)
+                    tma_load_3d(sQ + t * F::QBytes + c * kChunkBytes, &tm_q, &ctl->q_full, 0, (int)n0,
+                                (b * Hq + h0 + t) * C + c);
             bool ok = true;
             for (int j = 0; j < nkt && ok; ++j) {
-                const int st = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
+                const int ks = j % KS, vs = j % VS;
                 const int64_t m0 = (int64_t)j * kBN;
-                const Band bd = tile_band(w, H, n0, m0);
-                const int ca = bd.r_lo >> 3;
+                const int ca = tile_band(w, H, n0, m0).r_lo >> 3;
                 wc.site = 1;
-                if (!(ok = mbar_wait(&ctl->k_empty[st], ph ^ 1, wc))) break;
-                mbar_expect_tx(&ctl->k_full[st], (uint32_t)(C - ca) * kChunkBytes);
+                if (!(ok = mbar_wait(&ctl->k_empty[ks], ((j / KS) & 1) ^ 1, wc))) break;
+                mbar_expect_tx(&ctl->k_full[ks], (uint32_t)(C - ca) * kChunkBytes);
                 for (int c = ca; c < C; ++c)
-                    tma_load_3d(sK + st * L::KBytes + c * kChunkBytes, &tm_k, &ctl->k_full[st], 0, (int)m0,
+                    tma_load_3d(sK + ks * F::KBytes + c * kChunkBytes, &tm_k, &ctl->k_full[ks], 0, (int)m0,
                                 (b * Hkv + kvh) * C + c);
-                last_k[st] = j;
+                last_k[ks] = j;
                 wc.site = 2;
-                if (!(ok = mbar_wait(&ctl->v_empty[st], ph ^ 1, wc))) break;
-                mbar_expect_tx(&ctl->v_full[st], L::VBytes);
+                if (!(ok = mbar_wait(&ctl->v_empty[vs], ((j / VS) & 1) ^ 1, wc))) break;
+                mbar_expect_tx(&ctl->v_full[vs], F::VBytes);
                 for (int gidx = 0; gidx < D / 64; ++gidx)
-                    tma_load_4d(sV + st * L::VBytes + gidx * 16384, &tm_v, &ctl->v_full[st], gidx * 64, kvh,
+                    tma_load_4d(sV + vs * F::VBytes + gidx * 16384, &tm_v, &ctl->v_full[vs], gidx * 64, kvh,
                                 (int)m0, b);
-                last_v[st] = j;
+                last_v[vs] = j;
             }
             if (!ok) {
                 // Let every copy this thread started land before the CTA exits.
                 wait_drain(&ctl->q_full, 0, limit_ns);
-                for (int s = 0; s < kStages; ++s) {
-                    if (last_k[s] >= 0) wait_drain(&ctl->k_full[s], (last_k[s] >> 1) & 1, limit_ns);
-                    if (last_v[s] >= 0) wait_drain(&ctl->v_full[s], (last_v[s] >> 1) & 1, limit_ns);
-                }
+                for (int s = 0; s < KS; ++s)
+                    if (last_k[s] >= 0) wait_drain(&ctl->k_full[s], (last_k[s] / KS) & 1, limit_ns);
+                for (int s = 0; s < VS; ++s)
+                    if (last_v[s] >= 0) wait_drain(&ctl->v_full[s], (last_v[s] / VS) & 1, limit_ns);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kWarpFix) {
+        // --------------------------------------------- pruned-pair zeroing
+        bool ok = true;
+        for (int j = 0; j < nkt && ok; ++j) {
+            const int ks = j % KS;
+            const int r_lo = tile_band(w, H, n0, (int64_t)j * kBN).r_lo;
+            const int ca = r_lo >> 3;
+            wc.site = 3;
+            if (!(ok = mbar_wait_warp(&ctl->k_full[ks], (j / KS) & 1, wc))) break;
+            if ((r_lo & 7) && ca < C) {
+                // Pairs [8*ca, r_lo) are pruned for every cell of this tile: zero them
+                // in the landed K~ chunk so the dense MMA over whole chunks skips them.
+                uint8_t *chunk = sK + ks * F::KBytes + ca * kChunkBytes;
+                for (int row = lane; row < kBN; row += 32)
+                    for (int p = 0; p < (r_lo & 7); ++p)
+                        *reinterpret_cast<uint32_t *>(chunk + sw32_off(row, p)) = 0u;
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->k_ready[ks]);
+        }
+    } else if (warp == kWarpMma) {
         // ---------------------------------------------------------- MMA issuer
         const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
         const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
-        const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
-        bool ok = true;
-        wc.site = 3;
-        ok = mbar_wait_warp(&ctl->q_full, 0, wc);
-        auto issue_pv = [&](int jj) -> bool {
-            const int st = jj & 1;
-            wc.site = 4;
-            if (!mbar_wait_warp(&ctl->v_full[st], (jj >> 1) & 1, wc)) return false;
+        const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+        wc.site = 4;
+        bool ok = mbar_wait_warp(&ctl->q_full, 0, wc);
+        auto issue_qk = [&](int t, int ks, int ca) {
+            if (lane == 0) {
+                for (int c = ca; c < C; ++c) {
+                    const uint64_t da = smem_desc(sQa + t * F::QBytes + c * kChunkBytes, 16, 256, kSwizzle32B);
+                    const uint64_t db = smem_desc(sKa + ks * F::KBytes + c * kChunkBytes, 16, 256, kSwizzle32B);
+                    umma_bf16_ss(tmem + t * 128, da, db, idesc_qk, c > ca ? 1u : 0u);
+                }
+                umma_commit(&ctl->s_full[t]);
+            }
+            __syncwarp();
+        };
+        auto issue_pv = [&](int t, int jj, bool release_v) -> bool {
+            const int vs = jj % VS;
             wc.site = 5;
-            if (!mbar_wait_warp(&ctl->p_full, jj & 1, wc)) return false;
+            if (!mbar_wait_warp(&ctl->v_full[vs], (jj / VS) & 1, wc)) return false;
+            wc.site = 6;
+            if (!mbar_wait_warp(&ctl->p_full[t], jj & 1, wc)) return false;
             if (lane == 0) {
                 tc_fence_after();
+                const uint32_t o_col = t ? F::TmemO1 : F::TmemO0;
 #pragma unroll
-                for (int t = 0; t < kBN / 16; ++t) {
-                    // A = P keys [16t, 16t+16): K-major SW128, 64-key groups 16 KB apart.
-                    const uint64_t da = smem_desc(sPa + (t >> 2) * 16384 + (t & 3) * 32, 16, 1024, kSwizzle128B);
-                    // B = V rows [16t, 16t+16): MN-major SW128, 64-dim groups 16 KB apart.
-                    const uint64_t db =
-                        smem_desc(sVa + st * L::VBytes + t * 2048, 16384, 1024, kSwizzle128B);
-                    umma_bf16_ss(tmem + 256, da, db, idesc_pv, (jj > 0 || t > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kBN / 16; ++kk) {
+                    // A = P_t keys [16kk, 16kk+16): 8 TMEM columns of bf16 pairs.
+                    // B = V rows [16kk, 16kk+16): MN-major SW128, 64-dim groups 16 KB apart.
+                    const uint64_t db = smem_desc(sVa + vs * F::VBytes + kk * 2048, 16384, 1024, kSwizzle128B);
+                    umma_bf16_ts(tmem + o_col, tmem + t * 128 + kk * 8, db, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&ctl->o_ready);
-                umma_commit(&ctl->v_empty[st]);
+                umma_commit(&ctl->o_done[t]);
+                if (release_v) umma_commit(&ctl->v_empty[vs]);
             }
             __syncwarp();
             return true;
         };
         for (int j = 0; j < nkt && ok; ++j) {
-            const int st = j & 1, sb = j & 1;
-            const uint32_t ph = (j >> 1) & 1;
-            const Band bd = tile_band(w, H, (int64_t)qt * kBM, (int64_t)j * kBN);
-            const int ca = bd.r_lo >> 3;
-            wc.site = 6;
-            if (!(ok = mbar_wait_warp(&ctl->k_full[st], ph, wc))) break;
-            if ((bd.r_lo & 7) && ca < C) {
-                // Pairs [8*ca, r_lo) are pruned for every cell of this tile: zero them
-                // in the landed K~ chunk so the dense MMA over whole chunks skips them.
-                uint8_t *chunk = sK + st * L::KBytes + ca * kChunkBytes;
-                for (int row = lane; row < kBN; row += 32)
-                    for (int p = 8 * ca; p < bd.r_lo; ++p)
-                        *reinterpret_cast<uint32_t *>(chunk + sw32_off(row, p & 7)) = 0u;
-                fence_proxy_async_smem();
-            }
-            __syncwarp();
+            const int ks = j % KS;
+            const int ca = tile_band(w, H, n0, (int64_t)j * kBN).r_lo >> 3;
             wc.site = 7;
-            if (!(ok = mbar_wait_warp(&ctl->s_free[sb], ph ^ 1, wc))) break;
-            if (lane == 0) {
-                tc_fence_after();
-                for (int c = ca; c < C; ++c) {
-                    const uint64_t da = smem_desc(sQa + c * kChunkBytes, 16, 256, kSwizzle32B);
-                    const uint64_t db = smem_desc(sKa + st * L::KBytes + c * kChunkBytes, 16, 256, kSwizzle32B);
-                    umma_bf16_ss(tmem + sb * 128, da, db, idesc_qk, c > ca ? 1u : 0u);
-                }
-                umma_commit(&ctl->s_full[sb]);
-                umma_commit(&ctl->k_empty[st]);
-            }
+            if (!(ok = mbar_wait_warp(&ctl->k_ready[ks], (j / KS) & 1, wc))) break;
+            if (lane == 0) tc_fence_after();
+            issue_qk(0, ks, ca);
+            if (two && j > 0 && !(ok = issue_pv(1, j - 1, true))) break;
+            if (two) issue_qk(1, ks, ca);
+            if (lane == 0) umma_commit(&ctl->k_empty[ks]);
             __syncwarp();
-            if (j > 0 && !(ok = issue_pv(j - 1))) break;
+            if (!(ok = issue_pv(0, j, !two))) break;
         }
-        if (ok) ok = issue_pv(nkt - 1);
-    } else {
+        if (ok && two) ok = issue_pv(1, nkt - 1, true);
+    } else if (warp < 8) {
         // ------------------------------------------------------------- softmax
-        const int q4 = warp & 3;
-        const int row = q4 * 32 + lane;
-        const int64_t n = n0 + row;
-        const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
-        const float scale_log2 = 1.4426950408889634f * rsqrtf((float)D);
-        float mrun = -INFINITY, lrun = 0.f;
-        wc.site = 11;
-        bool ok = mbar_wait_warp(&ctl->q_full, 0, wc);  // Q~ rows are read for the boundary fix-up
-        for (int j = 0; j < nkt && ok; ++j) {
-            const int st = j & 1, sb = j & 1;
-            const uint32_t ph = (j >> 1) & 1;
-            const int64_t m0 = (int64_t)j * kBN;
-            const Band bd = tile_band(w, H, n0, m0);
-            float s[kBN];
+        const int t = warp >> 2;  // which head of the pair
+        if (t < nwg) {
+            const int q4 = warp & 3;
+            const int row = q4 * 32 + lane;
+            const int64_t n = n0 + row;
+            const int hq = h0 + t;
+            const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+            const uint32_t tS = tmem + (uint32_t)(t * 128) + lane_off;
+            const uint32_t tO = tmem + (t ? F::TmemO1 : F::TmemO0) + lane_off;
+            const uint8_t *sQt = sQ + t * F::QBytes;
+            const float scale_log2 = 1.4426950408889634f * rsqrtf((float)D);
+            float m_used = -INFINITY, lrun = 0.f;
             wc.site = 8;
-            if (!(ok = mbar_wait_warp(&ctl->s_full[sb], ph, wc))) break;
-            tc_fence_after();
-            if ((bd.r_lo >> 3) < C) {
+            bool ok = mbar_wait_warp(&ctl->q_full, 0, wc);  // Q~ rows are read for the boundary fix-up
+            for (int j = 0; j < nkt && ok; ++j) {
+                const int ks = j % KS;
+                const int64_t m0 = (int64_t)j * kBN;
+                const Band bd = tile_band(w, H, n0, m0);
+                float s[kBN];
+                wc.site = 9;
+                if (!(ok = mbar_wait_warp(&ctl->s_full[t], j & 1, wc))) break;
+                tc_fence_after();
+                if ((bd.r_lo >> 3) < C) {
+                    uint32_t r0[32], r1[32], r2[32], r3[32];
+                    tmem_ld_32x32b_x32(tS + 0, r0);
+                    tmem_ld_32x32b_x32(tS + 32, r1);
+                    tmem_ld_32x32b_x32(tS + 64, r2);
+                    tmem_ld_32x32b_x32(tS + 96, r3);
+                    tmem_ld_wait(r0);
+                    tmem_ld_wait(r1);
+                    tmem_ld_wait(r2);
+                    tmem_ld_wait(r3);
 #pragma unroll
-                for (int cc = 0; cc < kBN / 32; ++cc) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tl + sb * 128 + cc * 32, r);
-                    tmem_ld_wait(r);
+                    for (int i = 0; i < 32; ++i) {
+                        s[i] = __uint_as_float(r0[i]);
+                        s[32 + i] = __uint_as_float(r1[i]);
+                        s[64 + i] = __uint_as_float(r2[i]);
+                        s[96 + i] = __uint_as_float(r3[i]);
+                    }
+                } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < kBN; ++i) s[i] = 0.f;
                 }
-            } else {
+                // Boundary pairs: the dense MMA included them; remove them from the
+                // cells whose distance exceeds the pair's window (jj < n - m0 - w_r).
+                if (bd.r_lo < bd.r_full) {
+                    wc.site = 10;  // orders the landed K~ chunk before these reads
+                    if (!(ok = mbar_wait_warp(&ctl->k_full[ks], (j / KS) & 1, wc))) break;
+                    for (int r = bd.r_lo; r < bd.r_full; ++r) {
+                        const int lim = (int)(n - m0 - (int64_t)w[r]);
+                        const int lim_max = __reduce_max_sync(0xffffffffu, lim);
+                        if (lim_max <= 0) continue;
+                        const uint32_t qw =
+                            *reinterpret_cast<const uint32_t *>(sQt + (r >> 3) * kChunkBytes + sw32_off(row, r & 7));
+                        const float qa = bf16lo(qw), qb = bf16hi(qw);
+                        const uint8_t *kch = sK + ks * F::KBytes + (r >> 3) * kChunkBytes;
 #pragma unroll
-                for (int i = 0; i < kBN; ++i) s[i] = 0.f;
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->s_free[sb]);
-            // Boundary pairs: the dense MMA included them; remove them from the
-            // cells where the distance exceeds the pair's window.
-            if (bd.r_lo < bd.r_full) {
-                wc.site = 12;  // the K~ chunk landed long ago; this orders its TMA writes before our reads
-                if (!(ok = mbar_wait_warp(&ctl->k_full[st], ph, wc))) break;
-            }
-            for (int r = bd.r_lo; r < bd.r_full; ++r) {
-                const int64_t lim = n - m0 - (int64_t)w[r];  // cells jj < lim have n - m > w_r
-                if (lim > 0) {
-                    const uint32_t qw = *reinterpret_cast<const uint32_t *>(sQ + (r >> 3) * kChunkBytes +
-                                                                            sw32_off(row, r & 7));
-                    const float qa = bf16lo(qw), qb = bf16hi(qw);
-                    const uint8_t *kch = sK + st * L::KBytes + (r >> 3) * kChunkBytes;
+                        for (int cc = 0; cc < 4; ++cc) {
+                            if (32 * cc < lim_max) {
 #pragma unroll
-                    for (int jj = 0; jj < kBN; ++jj) {
-                        if (jj < lim) {
-                            const uint32_t kw = *reinterpret_cast<const uint32_t *>(kch + sw32_off(jj, r & 7));
-                            s[jj] -= qa * bf16lo(kw) + qb * bf16hi(kw);
+                                for (int i = 0; i < 32; ++i) {
+                                    const int jj = 32 * cc + i;
+                                    if (jj < lim) {
+                                        const uint32_t kw =
+                                            *reinterpret_cast<const uint32_t *>(kch + sw32_off(jj, r & 7));
+                                        s[jj] -= qa * bf16lo(kw) + qb * bf16hi(kw);
+                                    }
+                                }
+                            }
                         }
                     }
                 }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->k_empty[st]);
-            // Causal mask (diagonal tile only), scale to log2 units, running max.
-            float mx = mrun;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->k_empty[ks]);
+                // Scale to log2 units, causal mask on the diagonal tile, row max (4 chains).
+                const float2 sc2 = make_float2(scale_log2, scale_log2);
+                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+                const bool diag = (j == qt);
 #pragma unroll
-            for (int jj = 0; jj < kBN; ++jj) {
-                float x = s[jj] * scale_log2;
-                if (m0 + jj > n) x = -INFINITY;
-                s[jj] = x;
-                mx = fmaxf(mx, x);
-            }
-            const float alpha = fast_exp2(mrun - mx);
-            float rs = 0.f;
+                for (int jj = 0; jj < kBN; jj += 4) {
+                    float2 a = mul2(make_float2(s[jj], s[jj + 1]), sc2);
+                    float2 c = mul2(make_float2(s[jj + 2], s[jj + 3]), sc2);
+                    if (diag) {
+                        if (jj > row) a.x = -INFINITY;
+                        if (jj + 1 > row) a.y = -INFINITY;
+                        if (jj + 2 > row) c.x = -INFINITY;
+                        if (jj + 3 > row) c.y = -INFINITY;
+                    }
+                    s[jj] = a.x;
+                    s[jj + 1] = a.y;
+                    s[jj + 2] = c.x;
+                    s[jj + 3] = c.y;
+                    mx0 = fmaxf(mx0, a.x);
+                    mx1 = fmaxf(mx1, a.y);
+                    mx2 = fmaxf(mx2, c.x);
+                    mx3 = fmaxf(mx3, c.y);
+                }
+                const float tile_max = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+                // Keep the previous (stale) max unless the row max grew by more than
+                // 2^8: the final O / l uses the same max, so the result is exact.
+                const bool need = tile_max > m_used + kRescaleThreshold;
+                const float m_new = need ? tile_max : m_used;
+                const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
+                m_used = m_new;
+                // P = exp2(x - m) as bf16 pairs; S registers die as P is produced.
+                const float2 mneg = make_float2(-m_used, -m_used);
+                const float2 one2 = make_float2(1.f, 1.f);
+                float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
+                uint32_t pk[64];
 #pragma unroll
-            for (int jj = 0; jj < kBN; ++jj) {
-                const float p = fast_exp2(s[jj] - mx);
-                s[jj] = p;
-                rs += p;
-            }
-            lrun = lrun * alpha + rs;
-            mrun = mx;
-            if (j > 0) {
-                wc.site = 9;
-                if (!(ok = mbar_wait_warp(&ctl->o_ready, (j - 1) & 1, wc))) break;
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha < 1.f)) {
-#pragma unroll
+                for (int i = 0; i < 64; i += 2) {
+                    float2 xa = fma2(make_float2(s[2 * i], s[2 * i + 1]), one2, mneg);
+                    float2 xb = fma2(make_float2(s[2 * i + 2], s[2 * i + 3]), one2, mneg);
+                    xa.x = fast_exp2(xa.x);
+                    xa.y = fast_exp2(xa.y);
+                    xb.x = fast_exp2(xb.x);
+                    xb.y = fast_exp2(xb.y);
+                    l0 = add2(l0, xa);
+                    l1 = add2(l1, xb);
+                    pk[i] = pack_bf16x2(xa.x, xa.y);
+                    pk[i + 1] = pack_bf16x2(xb.x, xb.y);
+                }
+                // Rescale O only when some row's max grew past the threshold (rare).
+                if (j > 0 && __any_sync(0xffffffffu, need)) {
+                    wc.site = 11;
+                    if (!(ok = mbar_wait_warp(&ctl->o_done[t], (j - 1) & 1, wc))) break;
+                    tc_fence_after();
+#pragma unroll 1
                     for (int cc = 0; cc < D / 32; ++cc) {
                         uint32_t r[32];
-                        tmem_ld_32x32b_x32(tl + 256 + cc * 32, r);
+                        tmem_ld_32x32b_x32(tO + cc * 32, r);
                         tmem_ld_wait(r);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                        tmem_st_32x32b_x32(tl + 256 + cc * 32, r);
-                    }
-                    tmem_st_wait();
-                }
-            }
-            // P (bf16) to shared memory, K-major SW128: 64-key groups of 16 KB, 128 B rows.
-#pragma unroll
-            for (int kk = 0; kk < kBN / 8; ++kk) {
-                uint4 v4;
-                v4.x = pack_bf16x2(s[kk * 8 + 0], s[kk * 8 + 1]);
-                v4.y = pack_bf16x2(s[kk * 8 + 2], s[kk * 8 + 3]);
-                v4.z = pack_bf16x2(s[kk * 8 + 4], s[kk * 8 + 5]);
-                v4.w = pack_bf16x2(s[kk * 8 + 6], s[kk * 8 + 7]);
-                const uint32_t off = (uint32_t)(kk >> 3) * 16384u + (uint32_t)row * 128u +
-                                     ((((uint32_t)kk & 7u) ^ ((uint32_t)row & 7u)) << 4);
-                *reinterpret_cast<uint4 *>(sP + off) = v4;
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->p_full);
-        }
-        if (ok) {
-            wc.site = 10;
-            ok = mbar_wait_warp(&ctl->o_ready, (nkt - 1) & 1, wc);
-        }
-        if (ok) {
-            tc_fence_after();
-            const float inv = 1.f / lrun;
-            const size_t o = ((size_t)((int64_t)b * N + n) * Hq + hq) * D;
-#pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tl + 256 + cc * 32, r);
-                tmem_ld_wait(r);
-                if (n < N) {
-                    if (out_f32) {
-                        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + o + cc * 32);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                                                 __uint_as_float(r[4 * i + 2]) * inv,
-                                                 __uint_as_float(r[4 * i + 3]) * inv);
-                    } else {
-                        uint4 *dst =
-                            reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(out) + o + cc * 32);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(
-                                pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv),
-                                pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv),
-                                pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv),
-                                pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv));
+                        tmem_st_32x32b_x32(tO + cc * 32, r);
                     }
                 }
+                // P over the first 64 columns of S (S was read in full above).
+                {
+                    uint32_t (&pa)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
+                    uint32_t (&pb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
+                    tmem_st_32x32b_x32(tS + 0, pa);
+                    tmem_st_32x32b_x32(tS + 32, pb);
+                }
+                tmem_st_wait();
+                const float2 ls = add2(l0, l1);
+                lrun = lrun * alpha + (ls.x + ls.y);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->p_full[t]);
             }
-            if (lse && n < N) lse[((size_t)b * Hq + hq) * N + n] = (mrun + __log2f(lrun)) * 0.69314718055994531f;
+            if (ok) {
+                wc.site = 12;
+                ok = mbar_wait_warp(&ctl->o_done[t], (nkt - 1) & 1, wc);
+            }
+            if (ok) {
+                tc_fence_after();
+                const float inv = 1.f / lrun;
+                const size_t o = ((size_t)((int64_t)b * N + n) * Hq + hq) * D;
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tO + cc * 32, r);
+                    tmem_ld_wait(r);
+                    if (n < N) {
+                        if (out_f32) {
+                            float4 *dst =
+                                reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + o + cc * 32);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv,
+                                                     __uint_as_float(r[4 * i + 1]) * inv,
+                                                     __uint_as_float(r[4 * i + 2]) * inv,
+                                                     __uint_as_float(r[4 * i + 3]) * inv);
+                        } else {
+                            uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(out) + o +
+                                                                   cc * 32);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                dst[i] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv,
+                                                                __uint_as_float(r[8 * i + 1]) * inv),
+                                                    pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv,
+                                                                __uint_as_float(r[8 * i + 3]) * inv),
+                                                    pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv,
+                                                                __uint_as_float(r[8 * i + 5]) * inv),
+                                                    pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv,
+                                                                __uint_as_float(r[8 * i + 7]) * inv));
+                        }
+                    }
+                }
+                if (lse && n < N)
+                    lse[((size_t)b * Hq + hq) * N + n] = (m_used + __log2f(lrun)) * 0.69314718055994531f;
+            }
         }
     }
 
     // Teardown: every tensor-core operation must be complete before TMEM is freed.
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         if (lane == 0) {
             umma_commit(&ctl->drain);
             wait_drain(&ctl->drain, 0, limit_ns);
@@ -472,16 +551,17 @@ cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *
         if (e != cudaSuccess) return e;
     }
     const int num_qt = (int)((p.N + tc::kBM - 1) / tc::kBM);
-    dim3 grid((unsigned)num_qt, (unsigned)(p.B * p.Hq));
+    const int G = p.Hq / p.Hkv;
+    dim3 grid((unsigned)num_qt, (unsigned)(p.B * p.Hkv * ((G + 1) / 2)));
     cudaError_t e;
     if (p.D == 128) {
-        const int smem = tc::Layout<128>::Request;
+        const int smem = tc::Cfg<128>::Request;
         e = cudaFuncSetAttribute(tc::prefill_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         tc::prefill_tc_kernel<128><<<grid, tc::kThreads, smem, s>>>(tq, tk, tv, wp, out, out_f32, lse, p.N, p.Hq,
                                                                     p.Hkv, status, wait_limit_ns);
     } else if (p.D == 64) {
-        const int smem = tc::Layout<64>::Request;
+        const int smem = tc::Cfg<64>::Request;
         e = cudaFuncSetAttribute(tc::prefill_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         tc::prefill_tc_kernel<64><<<grid, tc::kThreads, smem, s>>>(tq, tk, tv, wp, out, out_f32, lse, p.N, p.Hq,
