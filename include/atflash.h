@@ -179,6 +179,27 @@ int atflash_decode(const void *q, const void *kcache, const void *vcache, const 
                    void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Decode that allocates nothing (no counterpart in the paper; an addition of
+ * this library).  For callers that cannot allocate device memory at the call
+ * site, e.g. a serving loop that must never enter the CUDA allocator once it
+ * is running, or a plugin whose host framework owns all device memory.  Same
+ * arguments and results as atflash_decode, without the workspace: the split
+ * states live in a fixed device array of ATFLASH_NOALLOC_SCRATCH_BYTES that
+ * every GPU loading the library reserves until the process exits.
+ *   Returns ATFLASH_ERR_WORKSPACE, launching nothing, when the problem needs
+ *   more than that (atflash_decode_workspace_bytes() > the limit).
+ *   Every call on a device shares the array: calls whose work overlaps on the
+ *   GPU race; calls on one stream are ordered.  The first call on a device
+ *   looks up the array's address with that device current; make it before any
+ *   stream capture begins.
+ */
+#define ATFLASH_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int atflash_decode_noalloc(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens,
+                           void *out, int B, int Hq, int Hkv, int64_t Nmax, int D, double rope_base,
+                           double k_window, int kcache_rotated, int kv_layout, int in_dtype, int out_dtype,
+                           cudaStream_t stream);
+
+/*
  * Device status word of the current device: ATFLASH_OK, or ATFLASH_ERR_TIMEOUT
  * when a kernel's bounded wait ran out since the last clear.  Synchronises
  * the device.  clear != 0 resets the word.
