@@ -29,10 +29,45 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "prefill tokens/s + decode µs/token vs N; % of bf16 TC / HBM roofline"
-WORKLOAD = {
-    "workload": "Qwen2.5-0.5B-shaped single-layer windowed prefill + decode of the last row",
-    "B": 1, "Hq": 14, "Hkv": 2, "D": 64, "N": 32768, "rope_base": 1e6, "k_window": 8.0, "seed": 1,
+
+
+def _pf(name, B, Hq, Hkv, D, N, base, k, seed):
+    return {"workload": name, "B": B, "Hq": Hq, "Hkv": Hkv, "D": D, "N": N, "rope_base": base, "k_window": k,
+            "seed": seed}
+
+
+# Prefill workloads: one step = RoPE pre-pass -> windowed prefill -> decode of the last row.
+WORKLOADS = {
+    "qwen05b_32k": _pf("Qwen2.5-0.5B-shaped single-layer windowed prefill + decode of the last row",
+                       1, 14, 2, 64, 32768, 1e6, 8.0, 1),
+    "llama3b_8k": _pf("Llama-3.2-3B-shaped single-layer windowed prefill + decode of the last row",
+                      1, 24, 8, 128, 8192, 5e5, 16.0, 2),
+    "llama3b_32k": _pf("Llama-3.2-3B-shaped single-layer windowed prefill + decode of the last row",
+                       1, 24, 8, 128, 32768, 5e5, 16.0, 2),
+    "llama3b_128k": _pf("Llama-3.2-3B-shaped single-layer windowed prefill + decode of the last row",
+                        1, 24, 8, 128, 131072, 5e5, 16.0, 2),
+    "qwen7b_256k": _pf("Qwen2.5-7B-1M-shaped single-layer windowed prefill + decode of the last row",
+                       1, 28, 4, 128, 262144, 1e7, 16.0, 3),
+    "qwen7b_256k_k64": _pf("Qwen2.5-7B-1M-shaped single-layer windowed prefill + decode of the last row",
+                           1, 28, 4, 128, 262144, 1e7, 64.0, 3),
+    "qwen7b_512k": _pf("Qwen2.5-7B-1M-shaped single-layer windowed prefill + decode of the last row",
+                       1, 28, 4, 128, 524288, 1e7, 16.0, 3),
+    "qwen7b_512k_k64": _pf("Qwen2.5-7B-1M-shaped single-layer windowed prefill + decode of the last row",
+                           1, 28, 4, 128, 524288, 1e7, 64.0, 3),
 }
+# Decode workloads: one step = one decode call (one token for each of B sequences).
+DECODE_WORKLOADS = {
+    "decode_1m": {"workload": "Qwen2.5-7B-1M-shaped decode, 4 sequences at 1M tokens", "B": 4, "Hq": 28,
+                  "Hkv": 4, "D": 128, "N": 1 << 20, "rope_base": 1e7, "k_window": 16.0, "seed": 4},
+    "decode_1m_k64": {"workload": "Qwen2.5-7B-1M-shaped decode, 4 sequences at 1M tokens", "B": 4, "Hq": 28,
+                      "Hkv": 4, "D": 128, "N": 1 << 20, "rope_base": 1e7, "k_window": 64.0, "seed": 4},
+    "decode_128k": {"workload": "Qwen2.5-7B-1M-shaped decode, 16 sequences at 128K tokens", "B": 16, "Hq": 28,
+                    "Hkv": 4, "D": 128, "N": 1 << 17, "rope_base": 1e7, "k_window": 16.0, "seed": 5},
+    "decode_128k_k64": {"workload": "Qwen2.5-7B-1M-shaped decode, 16 sequences at 128K tokens", "B": 16,
+                        "Hq": 28, "Hkv": 4, "D": 128, "N": 1 << 17, "rope_base": 1e7, "k_window": 64.0,
+                        "seed": 5},
+}
+WORKLOAD = WORKLOADS["qwen05b_32k"]
 L2_FLUSH_BYTES = 256 << 20
 KERNELS_PER_STEP = 5  # rope_pack(q), rope_pack(k), prefill_tc, decode_split, decode_merge
 
@@ -50,6 +85,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--workload", default="qwen05b_32k",
+                   choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS))
     p.add_argument("--N", type=int, default=None, help="override sequence length (sweeps)")
     p.add_argument("--k-window", type=float, default=None, help="override k (inf = window off)")
     return p.parse_args()
@@ -325,7 +362,7 @@ def run_ours(args, wl):
     achieved = flops / (kern_ms / 1e3) / 1e12
     traffic = TRAFFIC["bytes_per_launch"] if TRAFFIC["source_sha1"] == kernel_sha1() else None
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": "prefill_tc_kernel<64>",
+                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": f"prefill_tc_kernel<{D}>",
                 "kernel_ms": round(kern_ms, 4),
                 "peak_source": f"{src} ({'sustained' if long_region else 'burst'} bf16)",
                 "flops_per_launch": flops}
@@ -358,6 +395,69 @@ def run_ours(args, wl):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def decode_retained_bytes(atf, wl):
+    """Algorithmic bytes of one decode call: V in full, only the kept K elements,
+    the query and the output (bf16).  Kept K pairs over distances 0..L-1 of one
+    (sequence, KV head): sum_r (min(w_r, L-1) + 1)."""
+    B, Hq, Hkv, D, L = wl["B"], wl["Hq"], wl["Hkv"], wl["D"], wl["N"]
+    w = atf.window_table(D, wl["rope_base"], wl["k_window"], L)
+    kept_pairs = sum(min(x, L - 1) + 1 for x in w)
+    per_head = 2 * (D * L) + 2 * (2 * kept_pairs)
+    return B * Hkv * per_head + 2 * B * Hq * D * 2
+
+
+def run_decode(args, wl):
+    import torch
+    import long_context_attention_pair_b200 as atf
+    from long_context_attention_pair_b200 import synthetic
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, Hq, Hkv, D, L = wl["B"], wl["Hq"], wl["Hkv"], wl["D"], wl["N"]
+    base, kwin = wl["rope_base"], wl["k_window"]
+    q = synthetic.tensor_torch(wl["seed"], "q_dec", (B, Hq, D), "bf16", device=dev)
+    kc = synthetic.tensor_torch(wl["seed"], "k_cache", (B, Hkv, L, D), "bf16", device=dev)
+    vc = synthetic.tensor_torch(wl["seed"], "v_cache", (B, Hkv, L, D), "bf16", device=dev)
+    sl = torch.full((B,), L, dtype=torch.int32, device=dev)
+    out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(atf.decode_workspace_bytes(B, Hq, Hkv, L, D), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(kw, steps):
+        for _ in range(args.warmup):
+            atf.decode(q, kc, vc, sl, base, kw, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            atf.decode(q, kc, vc, sl, base, kw, out=out, workspace=ws)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ms = timed(kwin, args.steps)
+    clocks = sampler.stop()
+    ms_off = timed(math.inf, args.steps)
+    peaks, src = measured_peaks()
+    nbytes = decode_retained_bytes(atf, wl)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    line = {"metric": METRIC, "value": round(world * B / (ms / 1e3), 2), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(wl, l2="inputs larger than L2 (cache of %.1f GB)" % (2 * B * Hkv * L * D * 2 / 1e9)),
+            "decode": {"us_per_call": round(1e3 * ms, 2), "us_per_token": round(1e3 * ms / B, 2)},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                         "kernel": f"decode_tc_kernel<{D}> + decode_merge_kernel",
+                         "bytes_per_call": nbytes, "peak_source": src},
+            "window_off": {"ms_per_step": round(ms_off, 4), "us_per_token": round(1e3 * ms_off / B, 2)},
+            "on_off_speedup": round(ms_off / ms, 4), "gpu_launches": 2 * args.steps, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def e2e(atf, q, k, v, wl, args, dev, world):
@@ -409,7 +509,13 @@ def main():
     args = parse()
     if args.steps < 1 or args.warmup < 3:
         raise SystemExit("need --steps >= 1 and --warmup >= 3")
-    wl = dict(WORKLOAD)
+    if args.workload in DECODE_WORKLOADS:
+        wl = dict(DECODE_WORKLOADS[args.workload])
+        if args.k_window is not None:
+            wl["k_window"] = args.k_window
+        run_decode(args, wl)
+        return
+    wl = dict(WORKLOADS[args.workload])
     if args.N:
         wl["N"] = args.N
     if args.k_window is not None:

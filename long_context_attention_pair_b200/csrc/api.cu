@@ -20,7 +20,7 @@ static std::mutex g_mu;
 static int *g_status_ptr[64];
 static cudaMemPool_t g_pool[64];
 
-static int *status_word() {
+int *device_status_word() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     std::lock_guard<std::mutex> lk(g_mu);
@@ -67,7 +67,7 @@ EncodeTiledFn encode_tiled_fn() {
     return fn;
 }
 
-static uint64_t wait_limit_ns() {
+uint64_t wait_limit_ns() {
     static uint64_t v = 0;
     static std::once_flag once;
     std::call_once(once, [] {
@@ -169,7 +169,7 @@ static int run_prefill_packed(const void *qt, const void *kt, const void *v, voi
     const int out_f32 = (out_dtype == ATFLASH_F32);
     cudaError_t e;
     if (in_dtype == ATFLASH_BF16) {
-        int *status = status_word();
+        int *status = device_status_word();
         if (!status) return ATFLASH_ERR_CUDA;
         e = launch_prefill_tc(qt, kt, v, out, out_f32, lse, p, wp, status, wait_limit_ns(), stream);
     } else {
@@ -262,7 +262,7 @@ int atflash_prefill(const void *q, const void *k, const void *v, void *out, int 
 
 size_t atflash_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D) {
     if (check_shape(B, Hq, Hkv, Nmax) != ATFLASH_OK || (D != 64 && D != 128)) return 0;
-    return decode_workspace_bytes(B, Hq, Nmax, D);
+    return decode_workspace_bytes(B, Hq, Hkv, Nmax, D);
 }
 
 int atflash_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out,
@@ -282,7 +282,7 @@ int atflash_decode(const void *q, const void *kcache, const void *vcache, const 
     if (Hq / Hkv > 16) return ATFLASH_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out))
         return ATFLASH_ERR_ALIGNMENT;
-    const size_t need = decode_workspace_bytes(B, Hq, Nmax, D);
+    const size_t need = decode_workspace_bytes(B, Hq, Hkv, Nmax, D);
     if (!workspace || workspace_bytes < need) return ATFLASH_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 15u) return ATFLASH_ERR_ALIGNMENT;
     WindowParams wp;

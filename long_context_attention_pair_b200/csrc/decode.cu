@@ -1,5 +1,6 @@
-// Split-KV windowed decode: one query token per sequence over a contiguous
-// [B][Hkv][Nmax][D] cache ("Numbers"/"Using the ports": the window is a
+// Split-KV windowed decode, CUDA-core version (fp32 caches; the bf16 path is
+// the tensor-core kernel in decode_tc.cu): one query token per sequence over a
+// contiguous cache ("Numbers"/"Using the ports": the window is a
 // condition on which K elements are loaded).
 //
 // Kernel 1 (grid splits x Hkv x B): each CTA owns kSplitKeys consecutive cache
@@ -17,14 +18,27 @@
 
 namespace atf {
 
-constexpr int kSplitKeys = 2048;
 constexpr int kDecodeWarps = 4;
 constexpr int kMaxGroup = 16;  // query heads per KV head
 
-int decode_num_splits(int64_t Nmax) { return (int)((Nmax + kSplitKeys - 1) / kSplitKeys); }
+// Keys per split: enough (sequence, KV head, split) CTAs to fill 148 SMs twice,
+// a multiple of 256 keys, at most 4096.
+int decode_split_keys(int B, int Hkv, int64_t Nmax) {
+    const int64_t total = (int64_t)B * Hkv * Nmax;
+    int64_t per = (total + 295) / 296;
+    per = (per + 255) / 256 * 256;
+    if (per < 256) per = 256;
+    if (per > 4096) per = 4096;
+    return (int)per;
+}
 
-size_t decode_workspace_bytes(int B, int Hq, int64_t Nmax, int D) {
-    return (size_t)B * Hq * decode_num_splits(Nmax) * (D + 2) * sizeof(float);
+int decode_num_splits(int B, int Hkv, int64_t Nmax) {
+    const int sk = decode_split_keys(B, Hkv, Nmax);
+    return (int)((Nmax + sk - 1) / sk);
+}
+
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D) {
+    return (size_t)B * Hq * decode_num_splits(B, Hkv, Nmax) * (D + 2) * sizeof(float);
 }
 
 __device__ __forceinline__ float2 dec_cos_sin(int64_t n, double theta) {
@@ -51,7 +65,7 @@ __device__ __forceinline__ int dec_first_kept_pair(const int *w, int H, int64_t 
 template <typename T, int D>
 __global__ void __launch_bounds__(32 * kDecodeWarps) decode_split_kernel(
     const T *__restrict__ q, const T *__restrict__ kc, const T *__restrict__ vc, const int32_t *__restrict__ seqlens,
-    float *__restrict__ ws, int Hq, int Hkv, int64_t Nmax, int krot, int nhd, int nsplit,
+    float *__restrict__ ws, int Hq, int Hkv, int64_t Nmax, int krot, int nhd, int split_keys, int nsplit,
     const __grid_constant__ WindowParams wp) {
     constexpr int H = D / 2;
     constexpr int PPL = H / 32;  // pairs per lane
@@ -64,8 +78,8 @@ __global__ void __launch_bounds__(32 * kDecodeWarps) decode_split_kernel(
     const int G = Hq / Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t L = seqlens[b];
-    const int64_t s0 = (int64_t)split * kSplitKeys;
-    const int64_t s1 = (s0 + kSplitKeys < L) ? s0 + kSplitKeys : L;
+    const int64_t s0 = (int64_t)split * split_keys;
+    const int64_t s1 = (s0 + split_keys < L) ? s0 + split_keys : L;
     for (int r = tid; r < H; r += blockDim.x) sw[r] = wp.w[r];
     for (int e = tid; e < G * H; e += blockDim.x) {
         const int j = e / H, r = e % H;
@@ -192,21 +206,29 @@ __global__ void decode_merge_kernel(const float *__restrict__ ws, void *out, int
 cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const int32_t *seqlens, void *out,
                           int out_f32, int in_f32, int krot, int nhd, const Problem &p, const WindowParams &wp,
                           float *workspace, cudaStream_t s) {
-    const int nsplit = decode_num_splits(p.N);
-    dim3 grid((unsigned)nsplit, (unsigned)p.Hkv, (unsigned)p.B);
-    dim3 block(32 * kDecodeWarps);
-#define ATF_DEC(T, DD)                                                                                      \
-    decode_split_kernel<T, DD><<<grid, block, 0, s>>>((const T *)q, (const T *)kc, (const T *)vc, seqlens,  \
-                                                      workspace, p.Hq, p.Hkv, p.N, krot, nhd, nsplit, wp)
-    if (p.D == 128) {
-        if (in_f32) ATF_DEC(float, 128); else ATF_DEC(__nv_bfloat16, 128);
-    } else if (p.D == 64) {
-        if (in_f32) ATF_DEC(float, 64); else ATF_DEC(__nv_bfloat16, 64);
+    const int split_keys = decode_split_keys(p.B, p.Hkv, p.N);
+    const int nsplit = decode_num_splits(p.B, p.Hkv, p.N);
+    cudaError_t e;
+    if (!in_f32) {
+        int *status = device_status_word();
+        if (!status) return cudaErrorUnknown;
+        e = launch_decode_tc(q, kc, vc, seqlens, krot, nhd, p, wp, workspace, split_keys, nsplit, status,
+                             wait_limit_ns(), s);
     } else {
-        return cudaErrorInvalidValue;
+        dim3 grid((unsigned)nsplit, (unsigned)p.Hkv, (unsigned)p.B);
+        dim3 block(32 * kDecodeWarps);
+        if (p.D == 128)
+            decode_split_kernel<float, 128><<<grid, block, 0, s>>>((const float *)q, (const float *)kc,
+                                                                   (const float *)vc, seqlens, workspace, p.Hq,
+                                                                   p.Hkv, p.N, krot, nhd, split_keys, nsplit, wp);
+        else if (p.D == 64)
+            decode_split_kernel<float, 64><<<grid, block, 0, s>>>((const float *)q, (const float *)kc,
+                                                                  (const float *)vc, seqlens, workspace, p.Hq,
+                                                                  p.Hkv, p.N, krot, nhd, split_keys, nsplit, wp);
+        else
+            return cudaErrorInvalidValue;
+        e = cudaGetLastError();
     }
-#undef ATF_DEC
-    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     decode_merge_kernel<<<dim3((unsigned)p.Hq, (unsigned)p.B), (unsigned)p.D, 0, s>>>(workspace, out, out_f32,
                                                                                         p.Hq, nsplit, p.D);

@@ -79,7 +79,7 @@ extern "C" int atflash_decode_noalloc(const void *q, const void *kcache, const v
         return ATFLASH_ERR_UNSUPPORTED;
     if (Hq / Hkv > 16) return ATFLASH_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out)) return ATFLASH_ERR_ALIGNMENT;
-    if (decode_workspace_bytes(B, Hq, Nmax, D) > kScratchBytes) return ATFLASH_ERR_WORKSPACE;
+    if (decode_workspace_bytes(B, Hq, Hkv, Nmax, D) > kScratchBytes) return ATFLASH_ERR_WORKSPACE;
 
     WindowParams wp;
     int64_t w[kMaxPairs];

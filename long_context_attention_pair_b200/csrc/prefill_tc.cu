@@ -52,6 +52,14 @@ constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpFix = 10;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kChunkBytes = kBN * 32;  // 128 rows x 16 bf16 (one K-step)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
+// Of every 8 element pairs of a softmax row, this many take exp2 on the FMA
+// pipe (polynomial) and the rest on the multi-function unit, so that neither
+// unit alone bounds the softmax.
+constexpr int kPolyPairsOf8 = 0;
+// Boundary pairs whose key values the fix-up warp stages per tile (fp32, two
+// keys per 16 bytes); a tile with more boundary pairs handles the rest directly
+// from the K~ chunk.
+constexpr int kMaxStagedPairs = 8;
 
 template <int D>
 struct Cfg {
@@ -64,10 +72,15 @@ struct Cfg {
     static constexpr int OffQ = 0;                    // two query tiles
     static constexpr int OffK = OffQ + 2 * QBytes;
     static constexpr int OffV = OffK + KS * KBytes;
-    static constexpr int OffCtl = OffV + VS * VBytes;
+    static constexpr int OffBnd = OffV + VS * VBytes;                 // [KS][kMaxStagedPairs][64] float4
+    static constexpr int BndBytes = kMaxStagedPairs * 64 * 16;
+    static constexpr int OffCtl = OffBnd + KS * BndBytes;
     static constexpr int Total = OffCtl + 2048;
     static constexpr int Request = Total + 1024;
     static constexpr uint32_t TmemO0 = 256, TmemO1 = 256 + D;
+    // D = 64 leaves 128 TMEM columns for P of its own; D = 128 writes P over S.
+    static constexpr bool SepP = (D == 64);
+    static constexpr uint32_t TmemP0 = SepP ? 384 : 0, TmemP1 = SepP ? 448 : 128;
 };
 
 template <int KS, int VS>
@@ -75,7 +88,7 @@ struct Ctl {
     uint64_t q_full;
     uint64_t k_full[KS], k_ready[KS], k_empty[KS];
     uint64_t v_full[VS], v_empty[VS];
-    uint64_t s_full[2], p_full[2], o_done[2];
+    uint64_t s_full[2], s_read[2], p_full[2], o_done[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -110,6 +123,29 @@ __device__ __forceinline__ Band tile_band(const int *w, int H, int64_t n0, int64
     return b;
 }
 
+// The band of key tile j as j advances: both distances shrink by kBN per tile,
+// so r_lo and r_full only move down; each step is amortised O(1) instead of a
+// binary search on the critical path.
+struct BandWalk {
+    int r_lo, r_full;
+    __device__ __forceinline__ void init(const int *w, int H, int64_t n0) {
+        const Band b = tile_band(w, H, n0, 0);
+        r_lo = b.r_lo;
+        r_full = b.r_full;
+    }
+    __device__ __forceinline__ Band at(const int *w, int64_t n0, int64_t m0) {
+        int64_t dmin = n0 - (m0 + kBN - 1);
+        if (dmin < 0) dmin = 0;
+        const int64_t dmax = n0 + kBM - 1 - m0;
+        while (r_lo > 0 && (int64_t)w[r_lo - 1] >= dmin) --r_lo;
+        while (r_full > 0 && (int64_t)w[r_full - 1] >= dmax) --r_full;
+        Band b;
+        b.r_lo = r_lo;
+        b.r_full = r_full;
+        return b;
+    }
+};
+
 __device__ __forceinline__ bool wait_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
@@ -133,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sQ = smem + F::OffQ;
     uint8_t *sK = smem + F::OffK;
     uint8_t *sV = smem + F::OffV;
+    float4 *sBnd = reinterpret_cast<float4 *>(smem + F::OffBnd);
     Ctl<KS, VS> *ctl = reinterpret_cast<Ctl<KS, VS> *>(smem + F::OffCtl);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -163,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&ctl->s_full[s], 1);
+            mbar_init(&ctl->s_read[s], 4);
             mbar_init(&ctl->p_full[s], 4);
             mbar_init(&ctl->o_done[s], 1);
         }
@@ -182,6 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int *w = ctl->w;
     WaitCtl wc{&ctl->abort_flag, status, limit_ns, 0};
 
+    // Register split: the launch gives every thread 168 registers (384 x 168 =
+    // 64512).  Warpgroup 2 (producer, fix-up, MMA, idle) drops to 96 and the two
+    // softmax warpgroups rise to 200: 128 x 96 + 256 x 200 = 63488 <= 64512.
+    if (warp >= 8) setmaxnreg_dec<96>();
     if (warp == kWarpProducer) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -197,10 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_3d(sQ + t * F::QBytes + c * kChunkBytes, &tm_q, &ctl->q_full, 0, (int)n0,
                                 (b * Hq + h0 + t) * C + c);
             bool ok = true;
+            BandWalk bw;
+            bw.init(w, H, n0);
             for (int j = 0; j < nkt && ok; ++j) {
                 const int ks = j % KS, vs = j % VS;
                 const int64_t m0 = (int64_t)j * kBN;
-                const int ca = tile_band(w, H, n0, m0).r_lo >> 3;
+                const int ca = bw.at(w, n0, m0).r_lo >> 3;
                 wc.site = 1;
                 if (!(ok = mbar_wait(&ctl->k_empty[ks], ((j / KS) & 1) ^ 1, wc))) break;
                 mbar_expect_tx(&ctl->k_full[ks], (uint32_t)(C - ca) * kChunkBytes);
@@ -226,21 +270,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == kWarpFix) {
-        // --------------------------------------------- pruned-pair zeroing
+        // ------------------------- pruned-pair zeroing and boundary staging
         bool ok = true;
+        BandWalk bw;
+        bw.init(w, H, n0);
         for (int j = 0; j < nkt && ok; ++j) {
             const int ks = j % KS;
-            const int r_lo = tile_band(w, H, n0, (int64_t)j * kBN).r_lo;
+            const Band bd = bw.at(w, n0, (int64_t)j * kBN);
+            const int r_lo = bd.r_lo;
             const int ca = r_lo >> 3;
             wc.site = 3;
             if (!(ok = mbar_wait_warp(&ctl->k_full[ks], (j / KS) & 1, wc))) break;
+            // Boundary pairs r_lo + b: key values of keys (2i, 2i+1) as
+            // (k_r[2i], k_r[2i+1], k_{r+H}[2i], k_{r+H}[2i+1]) in fp32.
+            const int nb = min(bd.r_full - r_lo, kMaxStagedPairs);
+            float4 *bst = sBnd + ks * (kMaxStagedPairs * 64);
+            for (int e = lane; e < nb * 64; e += 32) {
+                const int bi = e >> 6, i = e & 63, r = r_lo + bi;
+                const uint8_t *kch = sK + ks * F::KBytes + (r >> 3) * kChunkBytes;
+                const uint32_t w0 = *reinterpret_cast<const uint32_t *>(kch + sw32_off(2 * i, r & 7));
+                const uint32_t w1 = *reinterpret_cast<const uint32_t *>(kch + sw32_off(2 * i + 1, r & 7));
+                bst[e] = make_float4(bf16lo(w0), bf16lo(w1), bf16hi(w0), bf16hi(w1));
+            }
             if ((r_lo & 7) && ca < C) {
                 // Pairs [8*ca, r_lo) are pruned for every cell of this tile: zero them
                 // in the landed K~ chunk so the dense MMA over whole chunks skips them.
+                // Lane -> (row, word) with consecutive lanes on consecutive words.
                 uint8_t *chunk = sK + ks * F::KBytes + ca * kChunkBytes;
-                for (int row = lane; row < kBN; row += 32)
-                    for (int p = 0; p < (r_lo & 7); ++p)
-                        *reinterpret_cast<uint32_t *>(chunk + sw32_off(row, p)) = 0u;
+                const int z = r_lo & 7;
+#pragma unroll 4
+                for (int e = lane; e < kBN * 8; e += 32)
+                    if ((e & 7) < z) *reinterpret_cast<uint32_t *>(chunk + sw32_off(e >> 3, e & 7)) = 0u;
                 fence_proxy_async_smem();
             }
             __syncwarp();
@@ -278,7 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // A = P_t keys [16kk, 16kk+16): 8 TMEM columns of bf16 pairs.
                     // B = V rows [16kk, 16kk+16): MN-major SW128, 64-dim groups 16 KB apart.
                     const uint64_t db = smem_desc(sVa + vs * F::VBytes + kk * 2048, 16384, 1024, kSwizzle128B);
-                    umma_bf16_ts(tmem + o_col, tmem + t * 128 + kk * 8, db, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                    umma_bf16_ts(tmem + o_col, tmem + (t ? F::TmemP1 : F::TmemP0) + kk * 8, db, idesc_pv,
+                                 (jj > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&ctl->o_done[t]);
                 if (release_v) umma_commit(&ctl->v_empty[vs]);
@@ -286,22 +347,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             return true;
         };
+        BandWalk bw;
+        bw.init(w, H, n0);
         for (int j = 0; j < nkt && ok; ++j) {
             const int ks = j % KS;
-            const int ca = tile_band(w, H, n0, (int64_t)j * kBN).r_lo >> 3;
+            const int ca = bw.at(w, n0, (int64_t)j * kBN).r_lo >> 3;
             wc.site = 7;
             if (!(ok = mbar_wait_warp(&ctl->k_ready[ks], (j / KS) & 1, wc))) break;
             if (lane == 0) tc_fence_after();
-            issue_qk(0, ks, ca);
-            if (two && j > 0 && !(ok = issue_pv(1, j - 1, true))) break;
-            if (two) issue_qk(1, ks, ca);
-            if (lane == 0) umma_commit(&ctl->k_empty[ks]);
-            __syncwarp();
-            if (!(ok = issue_pv(0, j, !two))) break;
+            if constexpr (F::SepP) {
+                // S_t(j) as soon as softmax t has read S_t(j-1); PV of the previous
+                // tile follows once its P is written.
+                wc.site = 13;
+                if (j > 0 && !(ok = mbar_wait_warp(&ctl->s_read[0], (j - 1) & 1, wc))) break;
+                if (lane == 0) tc_fence_after();
+                issue_qk(0, ks, ca);
+                if (two) {
+                    if (j > 0 && !(ok = mbar_wait_warp(&ctl->s_read[1], (j - 1) & 1, wc))) break;
+                    if (lane == 0) tc_fence_after();
+                    issue_qk(1, ks, ca);
+                }
+                if (lane == 0) umma_commit(&ctl->k_empty[ks]);
+                __syncwarp();
+                if (j > 0) {
+                    if (!(ok = issue_pv(0, j - 1, !two))) break;
+                    if (two && !(ok = issue_pv(1, j - 1, true))) break;
+                }
+            } else {
+                // P_t is written over S_t: S_t(j) only after PV_t(j-1) was issued.
+                issue_qk(0, ks, ca);
+                if (two && j > 0 && !(ok = issue_pv(1, j - 1, true))) break;
+                if (two) issue_qk(1, ks, ca);
+                if (lane == 0) umma_commit(&ctl->k_empty[ks]);
+                __syncwarp();
+                if (!(ok = issue_pv(0, j, !two))) break;
+            }
+        }
+        if constexpr (F::SepP) {
+            if (ok) ok = issue_pv(0, nkt - 1, !two);
         }
         if (ok && two) ok = issue_pv(1, nkt - 1, true);
     } else if (warp < 8) {
         // ------------------------------------------------------------- softmax
+        setmaxnreg_inc<200>();
         const int t = warp >> 2;  // which head of the pair
         if (t < nwg) {
             const int q4 = warp & 3;
@@ -310,16 +398,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int hq = h0 + t;
             const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
             const uint32_t tS = tmem + (uint32_t)(t * 128) + lane_off;
+            const uint32_t tP = tmem + (t ? F::TmemP1 : F::TmemP0) + lane_off;
             const uint32_t tO = tmem + (t ? F::TmemO1 : F::TmemO0) + lane_off;
             const uint8_t *sQt = sQ + t * F::QBytes;
             const float scale_log2 = 1.4426950408889634f * rsqrtf((float)D);
             float m_used = -INFINITY, lrun = 0.f;
             wc.site = 8;
             bool ok = mbar_wait_warp(&ctl->q_full, 0, wc);  // Q~ rows are read for the boundary fix-up
+            BandWalk bw;
+            bw.init(w, H, n0);
             for (int j = 0; j < nkt && ok; ++j) {
                 const int ks = j % KS;
                 const int64_t m0 = (int64_t)j * kBN;
-                const Band bd = tile_band(w, H, n0, m0);
+                const Band bd = bw.at(w, n0, m0);
                 float s[kBN];
                 wc.site = 9;
                 if (!(ok = mbar_wait_warp(&ctl->s_full[t], j & 1, wc))) break;
@@ -345,29 +436,70 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < kBN; ++i) s[i] = 0.f;
                 }
+                if constexpr (F::SepP) {
+                    // S_t(j) is in registers: the MMA may overwrite it with S_t(j+1).
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ctl->s_read[t]);
+                }
                 // Boundary pairs: the dense MMA included them; remove them from the
                 // cells whose distance exceeds the pair's window (jj < n - m0 - w_r).
                 if (bd.r_lo < bd.r_full) {
-                    wc.site = 10;  // orders the landed K~ chunk before these reads
-                    if (!(ok = mbar_wait_warp(&ctl->k_full[ks], (j / KS) & 1, wc))) break;
+                    wc.site = 10;  // the fix-up warp has staged this tile's boundary pairs
+                    if (!(ok = mbar_wait_warp(&ctl->k_ready[ks], (j / KS) & 1, wc))) break;
+                    const float4 *bst = sBnd + ks * (kMaxStagedPairs * 64);
                     for (int r = bd.r_lo; r < bd.r_full; ++r) {
                         const int lim = (int)(n - m0 - (int64_t)w[r]);
                         const int lim_max = __reduce_max_sync(0xffffffffu, lim);
                         if (lim_max <= 0) continue;
+                        const int lim_min = __reduce_min_sync(0xffffffffu, lim);
                         const uint32_t qw =
                             *reinterpret_cast<const uint32_t *>(sQt + (r >> 3) * kChunkBytes + sw32_off(row, r & 7));
-                        const float qa = bf16lo(qw), qb = bf16hi(qw);
-                        const uint8_t *kch = sK + ks * F::KBytes + (r >> 3) * kChunkBytes;
+                        const float2 qa2 = make_float2(bf16lo(qw), bf16lo(qw));
+                        const float2 qb2 = make_float2(bf16hi(qw), bf16hi(qw));
+                        if (r - bd.r_lo < kMaxStagedPairs) {
+                            const float4 *kb = bst + (r - bd.r_lo) * 64;
 #pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) {
-                            if (32 * cc < lim_max) {
+                            for (int cc = 0; cc < 4; ++cc) {
+                                if (32 * cc + 31 < lim_min) {
+                                    // Every row of the warp prunes the whole chunk.
 #pragma unroll
-                                for (int i = 0; i < 32; ++i) {
-                                    const int jj = 32 * cc + i;
-                                    if (jj < lim) {
-                                        const uint32_t kw =
-                                            *reinterpret_cast<const uint32_t *>(kch + sw32_off(jj, r & 7));
-                                        s[jj] -= qa * bf16lo(kw) + qb * bf16hi(kw);
+                                    for (int i = 0; i < 16; ++i) {
+                                        const float4 kv = kb[16 * cc + i];
+                                        const float2 t = fma2(qa2, make_float2(kv.x, kv.y),
+                                                              mul2(qb2, make_float2(kv.z, kv.w)));
+                                        const float2 r2 = add2(make_float2(s[32 * cc + 2 * i], s[32 * cc + 2 * i + 1]),
+                                                               make_float2(-t.x, -t.y));
+                                        s[32 * cc + 2 * i] = r2.x;
+                                        s[32 * cc + 2 * i + 1] = r2.y;
+                                    }
+                                } else if (32 * cc < lim_max) {
+#pragma unroll
+                                    for (int i = 0; i < 16; ++i) {
+                                        const int jj = 32 * cc + 2 * i;
+                                        const float4 kv = kb[16 * cc + i];
+                                        const float2 t = fma2(qa2, make_float2(kv.x, kv.y),
+                                                              mul2(qb2, make_float2(kv.z, kv.w)));
+                                        if (jj < lim) s[jj] -= t.x;
+                                        if (jj + 1 < lim) s[jj + 1] -= t.y;
+                                    }
+                                }
+                            }
+                        } else {
+                            // More boundary pairs than staged: read the K~ chunk directly.
+                            const float qa = qa2.x, qb = qb2.x;
+                            const uint8_t *kch = sK + ks * F::KBytes + (r >> 3) * kChunkBytes;
+#pragma unroll
+                            for (int cc = 0; cc < 4; ++cc) {
+                                if (32 * cc < lim_max) {
+#pragma unroll
+                                    for (int i = 0; i < 32; ++i) {
+                                        const int jj = 32 * cc + i;
+                                        if (jj < lim) {
+                                            const uint32_t kw =
+                                                *reinterpret_cast<const uint32_t *>(kch + sw32_off(jj, r & 7));
+                                            s[jj] -= qa * bf16lo(kw) + qb * bf16hi(kw);
+                                        }
                                     }
                                 }
                             }
@@ -376,59 +508,63 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->k_empty[ks]);
-                // Scale to log2 units, causal mask on the diagonal tile, row max (4 chains).
-                const float2 sc2 = make_float2(scale_log2, scale_log2);
-                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-                const bool diag = (j == qt);
+                // Causal mask on the diagonal tile; row max of the raw scores (4 chains
+                // of 3-input max); the 1/sqrt(D) * log2(e) scale is folded into the exp.
+                if (j == qt) {
 #pragma unroll
-                for (int jj = 0; jj < kBN; jj += 4) {
-                    float2 a = mul2(make_float2(s[jj], s[jj + 1]), sc2);
-                    float2 c = mul2(make_float2(s[jj + 2], s[jj + 3]), sc2);
-                    if (diag) {
-                        if (jj > row) a.x = -INFINITY;
-                        if (jj + 1 > row) a.y = -INFINITY;
-                        if (jj + 2 > row) c.x = -INFINITY;
-                        if (jj + 3 > row) c.y = -INFINITY;
-                    }
-                    s[jj] = a.x;
-                    s[jj + 1] = a.y;
-                    s[jj + 2] = c.x;
-                    s[jj + 3] = c.y;
-                    mx0 = fmaxf(mx0, a.x);
-                    mx1 = fmaxf(mx1, a.y);
-                    mx2 = fmaxf(mx2, c.x);
-                    mx3 = fmaxf(mx3, c.y);
+                    for (int jj = 0; jj < kBN; ++jj)
+                        if (jj > row) s[jj] = -INFINITY;
                 }
-                const float tile_max = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+                for (int jj = 0; jj < kBN; jj += 8) {
+                    mx0 = max3(mx0, s[jj], s[jj + 1]);
+                    mx1 = max3(mx1, s[jj + 2], s[jj + 3]);
+                    mx2 = max3(mx2, s[jj + 4], s[jj + 5]);
+                    mx3 = max3(mx3, s[jj + 6], s[jj + 7]);
+                }
+                const float tile_max = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * scale_log2;
                 // Keep the previous (stale) max unless the row max grew by more than
                 // 2^8: the final O / l uses the same max, so the result is exact.
                 const bool need = tile_max > m_used + kRescaleThreshold;
                 const float m_new = need ? tile_max : m_used;
                 const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
                 m_used = m_new;
-                // P = exp2(x - m) as bf16 pairs; S registers die as P is produced.
+                // P = exp2(s * scale - m) as bf16 pairs; S registers die as P is produced.
                 const float2 mneg = make_float2(-m_used, -m_used);
-                const float2 one2 = make_float2(1.f, 1.f);
+                const float2 sc2 = make_float2(scale_log2, scale_log2);
                 float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
                 uint32_t pk[64];
 #pragma unroll
                 for (int i = 0; i < 64; i += 2) {
-                    float2 xa = fma2(make_float2(s[2 * i], s[2 * i + 1]), one2, mneg);
-                    float2 xb = fma2(make_float2(s[2 * i + 2], s[2 * i + 3]), one2, mneg);
-                    xa.x = fast_exp2(xa.x);
-                    xa.y = fast_exp2(xa.y);
-                    xb.x = fast_exp2(xb.x);
-                    xb.y = fast_exp2(xb.y);
+                    float2 xa = fma2(make_float2(s[2 * i], s[2 * i + 1]), sc2, mneg);
+                    float2 xb = fma2(make_float2(s[2 * i + 2], s[2 * i + 3]), sc2, mneg);
+                    if (((i) & 7) < kPolyPairsOf8) {
+                        xa = exp2_fma2(xa);
+                    } else {
+                        xa.x = fast_exp2(xa.x);
+                        xa.y = fast_exp2(xa.y);
+                    }
+                    if (((i + 1) & 7) < kPolyPairsOf8) {
+                        xb = exp2_fma2(xb);
+                    } else {
+                        xb.x = fast_exp2(xb.x);
+                        xb.y = fast_exp2(xb.y);
+                    }
                     l0 = add2(l0, xa);
                     l1 = add2(l1, xb);
                     pk[i] = pack_bf16x2(xa.x, xa.y);
                     pk[i + 1] = pack_bf16x2(xb.x, xb.y);
                 }
                 // Rescale O only when some row's max grew past the threshold (rare).
-                if (j > 0 && __any_sync(0xffffffffu, need)) {
+                // With P in its own columns, PV_t(j-1) must also be done reading P.
+                const bool rescale = (j > 0) && __any_sync(0xffffffffu, need);
+                if (j > 0 && (F::SepP || rescale)) {
                     wc.site = 11;
                     if (!(ok = mbar_wait_warp(&ctl->o_done[t], (j - 1) & 1, wc))) break;
                     tc_fence_after();
+                }
+                if (rescale) {
 #pragma unroll 1
                     for (int cc = 0; cc < D / 32; ++cc) {
                         uint32_t r[32];
@@ -439,12 +575,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_st_32x32b_x32(tO + cc * 32, r);
                     }
                 }
-                // P over the first 64 columns of S (S was read in full above).
+                // P (its own columns, or the first 64 columns of S, read in full above).
                 {
                     uint32_t (&pa)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
                     uint32_t (&pb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-                    tmem_st_32x32b_x32(tS + 0, pa);
-                    tmem_st_32x32b_x32(tS + 32, pb);
+                    tmem_st_32x32b_x32(tP + 0, pa);
+                    tmem_st_32x32b_x32(tP + 32, pb);
                 }
                 tmem_st_wait();
                 const float2 ls = add2(l0, l1);

@@ -64,18 +64,29 @@ __device__ __forceinline__ void record_timeout(const WaitCtl &w) {
     atomicCAS(w.status, 0, ATFLASH_DEVICE_TIMEOUT_BASE + (int)w.site);
 }
 
+// try_wait that lets the hardware suspend the warp until the phase completes
+// (or `hint_ns` passes), so waiting warps do not spin on the issue slots their
+// busy neighbours need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.b32 %0, 1, 0, "
+        "p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const WaitCtl &w) {
     if (mbar_try_wait(bar, parity)) return true;
-    uint64_t t0 = globaltimer_ns();
-    uint32_t it = 0;
+    const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((++it & 255u) == 0) {
-            if (*w.abort_flag) return false;
-            if (globaltimer_ns() - t0 > w.limit_ns) {
-                record_timeout(w);
-                return false;
-            }
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+        if (*w.abort_flag) return false;
+        if (globaltimer_ns() - t0 > w.limit_ns) {
+            record_timeout(w);
+            return false;
         }
     }
 }
@@ -197,6 +208,17 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Per-warpgroup register budget changes (all four warps of a warpgroup execute
+// the same one).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------ descriptors
 // Shared-memory matrix descriptor (sm_100 format): start address, leading and
 // stride byte offsets (all >> 4), version 1 at bits 46-47, swizzle mode at 61-63.
@@ -248,6 +270,34 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     asm("mul.f32x2 %0, %1, %2;"
         : "=l"(reinterpret_cast<uint64_t &>(d))
         : "l"(reinterpret_cast<uint64_t const &>(a)), "l"(reinterpret_cast<uint64_t const &>(b)));
+    return d;
+}
+
+// exp2 of a pair on the FMA pipe.  Cody-Waite range reduction: n = round(x)
+// through the 1.5*2^23 magic add, f = x - n in [-1/2, 1/2]; 2^f by a degree-3
+// polynomial (weighted least-squares fit on Chebyshev nodes for relative error,
+// exact at f = 0; csrc/exp2_poly.py, max relative error 1.7e-4 in fp32); 2^n is
+// added to the exponent field: the integer n sits in the low mantissa bits of
+// x + 1.5*2^23, and shifting that word left by 23 leaves exactly n << 23.
+// Inputs are clamped to >= -125 (results below 2^-125 are far under bf16's
+// resolution of P; -inf maps to ~2^-125).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 magic = make_float2(12582912.f, 12582912.f);
+    const float2 t = add2(x, magic);
+    const float2 r = add2(t, make_float2(-12582912.f, -12582912.f));
+    const float2 f = fma2(r, make_float2(-1.f, -1.f), x);
+    float2 p = fma2(make_float2(0.055088684f, 0.055088684f), f, make_float2(0.24260405f, 0.24260405f));
+    p = fma2(p, f, make_float2(0.6932762f, 0.6932762f));
+    p = fma2(p, f, make_float2(1.f, 1.f));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
 

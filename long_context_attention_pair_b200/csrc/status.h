@@ -1,6 +1,6 @@
 // Status codes shared by the C ABI and the kernels.
 #pragma once
-#include "../../include/atflash.h"
+#include "atflash.h"
 
 // A kernel whose bounded wait ran out writes ATFLASH_DEVICE_TIMEOUT_BASE + site
 // into the device status word (first writer wins); the host maps any value at
