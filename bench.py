@@ -63,6 +63,15 @@ DECODE_WORKLOADS = {
                       "Hkv": 4, "D": 128, "N": 1 << 20, "rope_base": 1e7, "k_window": 64.0, "seed": 4},
     "decode_128k": {"workload": "Qwen2.5-7B-1M-shaped decode, 16 sequences at 128K tokens", "B": 16, "Hq": 28,
                     "Hkv": 4, "D": 128, "N": 1 << 17, "rope_base": 1e7, "k_window": 16.0, "seed": 5},
+    "decode_1m_packed": {"workload": "Qwen2.5-7B-1M-shaped decode, 4 sequences at 1M tokens, packed rotated K cache",
+                         "B": 4, "Hq": 28, "Hkv": 4, "D": 128, "N": 1 << 20, "rope_base": 1e7, "k_window": 16.0,
+                         "seed": 4, "packed": True},
+    "decode_1m_k64_packed": {"workload": "Qwen2.5-7B-1M-shaped decode, 4 sequences at 1M tokens, packed rotated K "
+                             "cache", "B": 4, "Hq": 28, "Hkv": 4, "D": 128, "N": 1 << 20, "rope_base": 1e7,
+                             "k_window": 64.0, "seed": 4, "packed": True},
+    "decode_128k_packed": {"workload": "Qwen2.5-7B-1M-shaped decode, 16 sequences at 128K tokens, packed rotated K "
+                           "cache", "B": 16, "Hq": 28, "Hkv": 4, "D": 128, "N": 1 << 17, "rope_base": 1e7,
+                           "k_window": 16.0, "seed": 5, "packed": True},
     "decode_128k_k64": {"workload": "Qwen2.5-7B-1M-shaped decode, 16 sequences at 128K tokens", "B": 16,
                         "Hq": 28, "Hkv": 4, "D": 128, "N": 1 << 17, "rope_base": 1e7, "k_window": 64.0,
                         "seed": 5},
@@ -424,15 +433,21 @@ def run_decode(args, wl):
     out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
     ws = torch.empty(atf.decode_workspace_bytes(B, Hq, Hkv, L, D), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    packed = bool(wl.get("packed"))
+    if packed:
+        # The RoPE pre-pass writes the rotated, chunk-major K cache once (not timed).
+        kc = atf.rope_pack(kc.permute(0, 2, 1, 3).contiguous(), base)
+        torch.cuda.synchronize()
+    dkw = dict(kcache_rotated=True, kv_layout="PACKED") if packed else {}
 
     def timed(kw, steps):
         for _ in range(args.warmup):
-            atf.decode(q, kc, vc, sl, base, kw, out=out, workspace=ws)
+            atf.decode(q, kc, vc, sl, base, kw, out=out, workspace=ws, **dkw)
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(steps):
-            atf.decode(q, kc, vc, sl, base, kw, out=out, workspace=ws)
+            atf.decode(q, kc, vc, sl, base, kw, out=out, workspace=ws, **dkw)
         b.record(stream)
         torch.cuda.synchronize()
         return a.elapsed_time(b) / steps

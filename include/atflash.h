@@ -57,6 +57,9 @@ typedef struct CUstream_st *cudaStream_t;
 /* KV-cache layouts accepted by atflash_decode. */
 #define ATFLASH_KV_HND 0 /* [B][Hkv][Nmax][D]: one contiguous block per (sequence, KV head) */
 #define ATFLASH_KV_NHD 1 /* [B][Nmax][Hkv][D]: token-major, the prefill's k/v layout */
+#define ATFLASH_KV_PACKED 2 /* K pre-rotated in atflash_rope_pack's bf16 layout [B*Hkv][D/16][Nmax][16]
+                               (8 frequency pairs per 32-byte chunk); V as [B][Hkv][Nmax][D].
+                               Pruned chunks are contiguous, so they are never fetched from HBM. */
 
 /* Text of a status code (static storage, never NULL). */
 const char *atflash_status_string(int status);
@@ -169,6 +172,7 @@ size_t atflash_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int 
  *                  of sequence b sits at position seqlens[b] - 1
  *   out            [B][Hq][D] written (out_dtype)
  *   kcache_rotated 0: keys are rotated on load; 1: keys already rotated
+ *                  (required by ATFLASH_KV_PACKED, which is bf16 only)
  *   in_dtype       element type of q, kcache, vcache (ATFLASH_BF16 or ATFLASH_F32)
  *   workspace      device buffer of >= atflash_decode_workspace_bytes(...) bytes
  *   D in {64, 128}.

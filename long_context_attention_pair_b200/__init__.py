@@ -25,6 +25,7 @@ F32 = 0
 BF16 = 1
 KV_HND = 0
 KV_NHD = 1
+KV_PACKED = 2
 OK = 0
 ERR_TIMEOUT = -5
 
@@ -217,7 +218,9 @@ def decode(q, k_cache, v_cache, seqlens, rope_base: float, k_window: float = mat
            kcache_rotated: bool = False, kv_layout: str = "HND", out=None, out_dtype=None, workspace=None,
            stream=None):
     """Windowed decode: q [B, Hq, D], seqlens int32 [B] (device), caches in
-    ``kv_layout`` "HND" [B, Hkv, Nmax, D] or "NHD" [B, Nmax, Hkv, D].
+    ``kv_layout`` "HND" [B, Hkv, Nmax, D], "NHD" [B, Nmax, Hkv, D], or "PACKED":
+    k_cache = ``rope_pack`` output [B*Hkv, D/16, Nmax, 16] (rotated; requires
+    ``kcache_rotated=True``) and v_cache [B, Hkv, Nmax, D].
 
     The query of sequence b sits at position seqlens[b] - 1.  Returns out [B, Hq, D].
     """
@@ -229,8 +232,11 @@ def decode(q, k_cache, v_cache, seqlens, rope_base: float, k_window: float = mat
     elif kv_layout == "NHD":
         _, Nmax, Hkv, _ = k_cache.shape
         lay = KV_NHD
+    elif kv_layout == "PACKED":
+        _, Hkv, Nmax, _ = v_cache.shape
+        lay = KV_PACKED
     else:
-        raise ValueError("kv_layout must be 'HND' or 'NHD'")
+        raise ValueError("kv_layout must be 'HND', 'NHD' or 'PACKED'")
     in_dtype = _dtype_code(q)
     if seqlens.dtype != torch.int32:
         raise TypeError("seqlens must be int32")

@@ -274,12 +274,15 @@ int atflash_decode(const void *q, const void *kcache, const void *vcache, const 
     if (rc != ATFLASH_OK) return rc;
     if ((rc = check_window_args(D, rope_base, k_window)) != ATFLASH_OK) return rc;
     if (kcache_rotated != 0 && kcache_rotated != 1) return ATFLASH_ERR_INVALID_ARG;
-    if (kv_layout != ATFLASH_KV_HND && kv_layout != ATFLASH_KV_NHD) return ATFLASH_ERR_INVALID_ARG;
+    if (kv_layout != ATFLASH_KV_HND && kv_layout != ATFLASH_KV_NHD && kv_layout != ATFLASH_KV_PACKED)
+        return ATFLASH_ERR_INVALID_ARG;
+    if (kv_layout == ATFLASH_KV_PACKED && !kcache_rotated) return ATFLASH_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
     if ((in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) ||
         (out_dtype != ATFLASH_F32 && out_dtype != ATFLASH_BF16))
         return ATFLASH_ERR_UNSUPPORTED;
     if (Hq / Hkv > 16) return ATFLASH_ERR_UNSUPPORTED;
+    if (kv_layout == ATFLASH_KV_PACKED && in_dtype != ATFLASH_BF16) return ATFLASH_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out))
         return ATFLASH_ERR_ALIGNMENT;
     const size_t need = decode_workspace_bytes(B, Hq, Hkv, Nmax, D);
@@ -289,7 +292,7 @@ int atflash_decode(const void *q, const void *kcache, const void *vcache, const 
     if ((rc = fill_window(wp, D, rope_base, k_window, Nmax)) != ATFLASH_OK) return rc;
     Problem p{B, Hq, Hkv, D, Nmax};
     cudaError_t e = launch_decode(q, kcache, vcache, seqlens, out, out_dtype == ATFLASH_F32,
-                                  in_dtype == ATFLASH_F32, kcache_rotated, kv_layout == ATFLASH_KV_NHD, p, wp,
+                                  in_dtype == ATFLASH_F32, kcache_rotated, kv_layout, p, wp,
                                   static_cast<float *>(workspace), stream);
     return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
 }

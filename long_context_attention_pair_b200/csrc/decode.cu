@@ -180,41 +180,83 @@ __global__ void __launch_bounds__(32 * kDecodeWarps) decode_split_kernel(
 }
 
 // Merge the per-split states (m in log2 units, l, unnormalised acc) of one
-// (sequence, query head) into the output row.
-__global__ void decode_merge_kernel(const float *__restrict__ ws, void *out, int out_f32, int Hq, int nsplit,
-                                    int D) {
-    const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+// (sequence, query head) into the output row: block-wide max and weighted sum
+// over the splits, then the accumulators summed by split-parallel thread groups.
+constexpr int kMergeThreads = 256;
+
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float *red) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float o = __shfl_xor_sync(0xffffffffu, v, off);
+        v = is_max ? fmaxf(v, o) : v + o;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    v = (lane < (int)(blockDim.x >> 5)) ? red[lane] : (is_max ? -INFINITY : 0.f);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float o = __shfl_xor_sync(0xffffffffu, v, off);
+        v = is_max ? fmaxf(v, o) : v + o;
+    }
+    return v;
+}
+
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float *__restrict__ ws, void *out,
+                                                                     int out_f32, int Hq, int nsplit, int D) {
+    __shared__ float red[32];
+    __shared__ float part_acc[kMergeThreads];
+    const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     const float *base = ws + ((size_t)b * Hq + h) * nsplit * (D + 2);
-    float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s)
-        if (base[(size_t)s * (D + 2) + 1] > 0.f) M = fmaxf(M, base[(size_t)s * (D + 2)]);
-    float l = 0.f, a = 0.f;
-    for (int s = 0; s < nsplit; ++s) {
+    float mx = -INFINITY;
+    for (int s = tid; s < nsplit; s += kMergeThreads) {
         const float *st = base + (size_t)s * (D + 2);
-        if (st[1] > 0.f) {
-            const float f = exp2f(st[0] - M);
-            l += st[1] * f;
-            a += st[2 + d] * f;
+        if (st[1] > 0.f) mx = fmaxf(mx, st[0]);
+    }
+    const float M = block_reduce(mx, true, red);
+    float ls = 0.f;
+    for (int s = tid; s < nsplit; s += kMergeThreads) {
+        const float *st = base + (size_t)s * (D + 2);
+        if (st[1] > 0.f) ls += st[1] * exp2f(st[0] - M);
+    }
+    const float Lsum = block_reduce(ls, false, red);
+    const int nparts = kMergeThreads / D, part = tid / D, d = tid % D;
+    float a = 0.f;
+    if (part < nparts) {
+#pragma unroll 4
+        for (int s = part; s < nsplit; s += nparts) {
+            const float *st = base + (size_t)s * (D + 2);
+            const float l = st[1];
+            if (l > 0.f) a += st[2 + d] * exp2f(st[0] - M);
         }
     }
-    const float val = a / l;
-    const size_t o = ((size_t)b * Hq + h) * D + d;
-    if (out_f32) reinterpret_cast<float *>(out)[o] = val;
-    else reinterpret_cast<__nv_bfloat16 *>(out)[o] = __float2bfloat16_rn(val);
+    part_acc[tid] = a;
+    __syncthreads();
+    if (tid < D) {
+        float acc = 0.f;
+        for (int pp = 0; pp < nparts; ++pp) acc += part_acc[pp * D + tid];
+        const float val = acc / Lsum;
+        const size_t o = ((size_t)b * Hq + h) * D + tid;
+        if (out_f32) reinterpret_cast<float *>(out)[o] = val;
+        else reinterpret_cast<__nv_bfloat16 *>(out)[o] = __float2bfloat16_rn(val);
+    }
 }
 
 cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const int32_t *seqlens, void *out,
-                          int out_f32, int in_f32, int krot, int nhd, const Problem &p, const WindowParams &wp,
+                          int out_f32, int in_f32, int krot, int layout, const Problem &p, const WindowParams &wp,
                           float *workspace, cudaStream_t s) {
+    const int nhd = (layout == ATFLASH_KV_NHD);
     const int split_keys = decode_split_keys(p.B, p.Hkv, p.N);
     const int nsplit = decode_num_splits(p.B, p.Hkv, p.N);
     cudaError_t e;
     if (!in_f32) {
         int *status = device_status_word();
         if (!status) return cudaErrorUnknown;
-        e = launch_decode_tc(q, kc, vc, seqlens, krot, nhd, p, wp, workspace, split_keys, nsplit, status,
+        e = launch_decode_tc(q, kc, vc, seqlens, krot, layout, p, wp, workspace, split_keys, nsplit, status,
                              wait_limit_ns(), s);
     } else {
+        if (layout == ATFLASH_KV_PACKED) return cudaErrorInvalidValue;  // packed caches are bf16
         dim3 grid((unsigned)nsplit, (unsigned)p.Hkv, (unsigned)p.B);
         dim3 block(32 * kDecodeWarps);
         if (p.D == 128)
@@ -230,7 +272,7 @@ cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const i
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<<<dim3((unsigned)p.Hq, (unsigned)p.B), (unsigned)p.D, 0, s>>>(workspace, out, out_f32,
+    decode_merge_kernel<<<dim3((unsigned)p.Hq, (unsigned)p.B), kMergeThreads, 0, s>>>(workspace, out, out_f32,
                                                                                         p.Hq, nsplit, p.D);
     return cudaGetLastError();
 }

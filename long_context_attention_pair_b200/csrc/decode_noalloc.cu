@@ -72,7 +72,10 @@ extern "C" int atflash_decode_noalloc(const void *q, const void *kcache, const v
     if ((int64_t)B * Hq > 65535 || !(rope_base > 1.0) || isnan(k_window) || k_window < 0.0)
         return ATFLASH_ERR_INVALID_ARG;
     if (kcache_rotated != 0 && kcache_rotated != 1) return ATFLASH_ERR_INVALID_ARG;
-    if (kv_layout != ATFLASH_KV_HND && kv_layout != ATFLASH_KV_NHD) return ATFLASH_ERR_INVALID_ARG;
+    if (kv_layout != ATFLASH_KV_HND && kv_layout != ATFLASH_KV_NHD && kv_layout != ATFLASH_KV_PACKED)
+        return ATFLASH_ERR_INVALID_ARG;
+    if (kv_layout == ATFLASH_KV_PACKED && (!kcache_rotated || in_dtype != ATFLASH_BF16))
+        return ATFLASH_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
     if ((in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) ||
         (out_dtype != ATFLASH_F32 && out_dtype != ATFLASH_BF16))
@@ -94,7 +97,6 @@ extern "C" int atflash_decode_noalloc(const void *q, const void *kcache, const v
     if ((rc = scratch_on_current_device(&scratch)) != ATFLASH_OK) return rc;
     Problem p{B, Hq, Hkv, D, Nmax};
     cudaError_t e = launch_decode(q, kcache, vcache, seqlens, out, out_dtype == ATFLASH_F32,
-                                  in_dtype == ATFLASH_F32, kcache_rotated, kv_layout == ATFLASH_KV_NHD, p, wp,
-                                  scratch, stream);
+                                  in_dtype == ATFLASH_F32, kcache_rotated, kv_layout, p, wp, scratch, stream);
     return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
 }

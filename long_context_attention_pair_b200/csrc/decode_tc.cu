@@ -17,6 +17,12 @@
 // Angles: the producer writes, per stage, the base angle stage_start*theta_r
 // reduced mod 2*pi in fp64; a key at offset i adds i*theta_r (i < 64) in fp32,
 // reduces once more and takes sin/cos on [-pi, pi].
+//
+// Packed cache (ATFLASH_KV_PACKED): K already rotated and stored as the RoPE
+// pre-pass writes it, [B*Hkv][D/16][Nmax][16] with 8 frequency pairs per 32-byte
+// chunk.  A pruned chunk of 64 keys is then 2 KB of HBM that is never fetched;
+// in the natural layouts a key's pruned dims are a short prefix of each 128-byte
+// half and HBM's access granularity fetches them anyway.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -27,13 +33,15 @@ namespace atf {
 namespace dtc {
 
 constexpr int kStageKeys = 64;
-constexpr int kStages = 3;
-constexpr int kConsumers = 4;
+constexpr int kWarpsPerStage = 4;                   // 16 keys per consumer warp
+constexpr int kGroups = 1;                          // groups consume stages round-robin
+constexpr int kConsumers = kWarpsPerStage * kGroups;
 constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr float kRescaleThreshold = 8.0f;
 
 template <int D>
 struct Cfg {
+    static constexpr int kStages = 3;
     static constexpr int H = D / 2;
     static constexpr int C = D / 16;                   // chunks of 8 pairs
     static constexpr int KBytes = C * 2 * 1024;        // [c][half][64 keys][8 dims] bf16
@@ -47,8 +55,9 @@ struct Cfg {
     static constexpr int Request = Total + 1024;
 };
 
+constexpr int kMaxStages = 8;
 struct Bars {
-    uint64_t full[kStages], empty[kStages];
+    uint64_t full[kMaxStages], empty[kMaxStages];
     int abort_flag;
 };
 
@@ -59,6 +68,13 @@ __device__ __forceinline__ int first_kept_pair(const int *w, int H, int64_t d) {
         if ((int64_t)w[mid] >= d) hi = mid; else lo = mid + 1;
     }
     return lo;
+}
+
+// r*(d) as d shrinks: keys of later stages are nearer the query, so the first
+// kept pair only moves down; amortised O(1) per stage.
+__device__ __forceinline__ int walk_down(const int *w, int r, int d) {
+    while (r > 0 && w[r - 1] >= d) --r;
+    return r;
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &d0, uint32_t &d1, uint32_t &d2, uint32_t &d3) {
@@ -97,13 +113,14 @@ __device__ __forceinline__ void mask_pairs(uint32_t &lo, uint32_t &hi, bool keep
     hi &= m;
 }
 
-template <int D>
+template <int D, bool kPacked>
 __global__ void __launch_bounds__(kThreads) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const void *q_,
     const int32_t *__restrict__ seqlens, float *__restrict__ ws, int Hq, int Hkv, int nhd, int krot, int split_keys,
     int nsplit, const __grid_constant__ WindowParams wp, int *status, uint64_t limit_ns) {
     using F = Cfg<D>;
     constexpr int H = F::H, C = F::C;
+    constexpr int kStages = F::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sK = smem + F::OffK;
@@ -126,7 +143,7 @@ __global__ void __launch_bounds__(kThreads) decode_tc_kernel(
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&bars->full[s], 1);
-            mbar_init(&bars->empty[s], kConsumers);
+            mbar_init(&bars->empty[s], kWarpsPerStage);
         }
         bars->abort_flag = 0;
         fence_mbar_init();
@@ -158,7 +175,8 @@ __global__ void __launch_bounds__(kThreads) decode_tc_kernel(
     if (warp == kConsumers) {
         // ------------------------------------------------------------ producer
         bool ok = true;
-        int last[kStages] = {-1, -1, -1};
+        int last[kMaxStages];
+        for (int s = 0; s < kMaxStages; ++s) last[s] = -1;
         for (int it = 0; it < nstage && ok; ++it) {
             const int st = it % kStages;
             const int64_t k0 = s0 + (int64_t)it * kStageKeys;
@@ -176,13 +194,18 @@ __global__ void __launch_bounds__(kThreads) decode_tc_kernel(
                 const uint32_t bytes = (uint32_t)(C - c_lo) * 2048u + (uint32_t)F::VBytes;
                 mbar_expect_tx(&bars->full[st], bytes);
                 uint8_t *kst = sK + st * F::KBytes;
-                for (int c = c_lo; c < C; ++c)
-                    for (int hf = 0; hf < 2; ++hf) {
-                        uint8_t *dst = kst + (2 * c + hf) * 1024;
-                        const int x = hf * H + 8 * c;
-                        if (nhd) tma_load_4d(dst, &tm_k, &bars->full[st], x, g, (int)k0, b);
-                        else tma_load_3d(dst, &tm_k, &bars->full[st], x, (int)k0, b * Hkv + g);
-                    }
+                if (kPacked) {
+                    for (int c = c_lo; c < C; ++c)
+                        tma_load_3d(kst + c * 2048, &tm_k, &bars->full[st], 0, (int)k0, (b * Hkv + g) * C + c);
+                } else {
+                    for (int c = c_lo; c < C; ++c)
+                        for (int hf = 0; hf < 2; ++hf) {
+                            uint8_t *dst = kst + (2 * c + hf) * 1024;
+                            const int x = hf * H + 8 * c;
+                            if (nhd) tma_load_4d(dst, &tm_k, &bars->full[st], x, g, (int)k0, b);
+                            else tma_load_3d(dst, &tm_k, &bars->full[st], x, (int)k0, b * Hkv + g);
+                        }
+                }
                 for (int gi = 0; gi < D / 64; ++gi) {
                     uint8_t *dst = sV + st * F::VBytes + gi * 8192;
                     if (nhd) tma_load_4d(dst, &tm_v, &bars->full[st], 64 * gi, g, (int)k0, b);
@@ -207,11 +230,20 @@ __global__ void __launch_bounds__(kThreads) decode_tc_kernel(
         uint32_t qa[C][4];
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            const int lo = 8 * c + 2 * tq, hi = H + 8 * c + 2 * tq;
-            qa[c][0] = pack_bf16x2(sQ[gq * D + lo], sQ[gq * D + lo + 1]);
-            qa[c][1] = pack_bf16x2(sQ[(gq + 8) * D + lo], sQ[(gq + 8) * D + lo + 1]);
-            qa[c][2] = pack_bf16x2(sQ[gq * D + hi], sQ[gq * D + hi + 1]);
-            qa[c][3] = pack_bf16x2(sQ[(gq + 8) * D + hi], sQ[(gq + 8) * D + hi + 1]);
+            if (kPacked) {
+                // k-order of a packed chunk: (pair 8c+e/2, component e%2).
+                const int pa = 8 * c + tq, pb = pa + 4;
+                qa[c][0] = pack_bf16x2(sQ[gq * D + pa], sQ[gq * D + pa + H]);
+                qa[c][1] = pack_bf16x2(sQ[(gq + 8) * D + pa], sQ[(gq + 8) * D + pa + H]);
+                qa[c][2] = pack_bf16x2(sQ[gq * D + pb], sQ[gq * D + pb + H]);
+                qa[c][3] = pack_bf16x2(sQ[(gq + 8) * D + pb], sQ[(gq + 8) * D + pb + H]);
+            } else {
+                const int lo = 8 * c + 2 * tq, hi = H + 8 * c + 2 * tq;
+                qa[c][0] = pack_bf16x2(sQ[gq * D + lo], sQ[gq * D + lo + 1]);
+                qa[c][1] = pack_bf16x2(sQ[(gq + 8) * D + lo], sQ[(gq + 8) * D + lo + 1]);
+                qa[c][2] = pack_bf16x2(sQ[gq * D + hi], sQ[gq * D + hi + 1]);
+                qa[c][3] = pack_bf16x2(sQ[(gq + 8) * D + hi], sQ[(gq + 8) * D + hi + 1]);
+            }
         }
         const float scale_log2 = 1.4426950408889634f * rsqrtf((float)D);
         float o[D / 8][4];
@@ -220,52 +252,89 @@ __global__ void __launch_bounds__(kThreads) decode_tc_kernel(
         float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};  // rows gq, gq+8
         const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
         bool ok = true;
-        for (int it = 0; it < nstage && ok; ++it) {
+        // Positions fit in int32 (Nmax <= 2^31 - 1).  Walk pointers for r*(d) of the
+        // stage's nearest key, this warp's nearest key and this warp's farthest key.
+        const int Lq = (int)L - 1;
+        int r_stage = H, r_warp = H, r_keep = H;
+        const int grp = warp / kWarpsPerStage, wq = warp % kWarpsPerStage;
+        for (int it = grp; it < nstage && ok; it += kGroups) {
             const int st = it % kStages;
-            const int64_t k0 = s0 + (int64_t)it * kStageKeys;
-            const int64_t kw0 = k0 + 16 * warp;  // this warp's first key
+            const int k0 = (int)s0 + it * kStageKeys;
+            const int kw0 = k0 + 16 * wq;  // this warp's first key
             if (!(ok = mbar_wait_warp(&bars->full[st], (it / kStages) & 1, wc))) break;
-            int64_t kw1 = kw0 + 15;
-            if (kw1 > s1 - 1) kw1 = s1 - 1;
-            int64_t k1 = k0 + kStageKeys - 1;
-            if (k1 > s1 - 1) k1 = s1 - 1;
-            const int c_stage = first_kept_pair(sw, H, (L - 1) - k1) >> 3;
+            const int kend = (int)s1 - 1;
+            const int kw1 = (kw0 + 15 < kend) ? kw0 + 15 : kend;
+            const int k1 = (k0 + kStageKeys - 1 < kend) ? k0 + kStageKeys - 1 : kend;
+            r_stage = walk_down(sw, r_stage, Lq - k1);
+            const int c_stage = r_stage >> 3;
             float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            if (kw0 < s1) {
-                const int c_warp = first_kept_pair(sw, H, (L - 1) - kw1) >> 3;
+            float sodd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            if (kw0 < (int)s1) {
+                r_warp = walk_down(sw, r_warp, Lq - kw1);
+                r_keep = walk_down(sw, r_keep, Lq - kw0);
+                const int c_warp = r_warp >> 3;
                 // Keys of this thread's fragments: n-tile 0 -> kw0 + gq, n-tile 1 -> kw0 + 8 + gq.
-                const int64_t key_a = kw0 + gq, key_b = kw0 + 8 + gq;
-                const int64_t da = (L - 1) - key_a, db = (L - 1) - key_b;
-                const float fa = (float)(16 * warp + gq), fb = fa + 8.f;
+                const int da = Lq - (kw0 + gq), db = da - 8;
+                const float fa = (float)(16 * wq + gq), fb = fa + 8.f;
                 const uint32_t kst = sKa + st * F::KBytes;
                 const int mi = lane >> 3, ri = lane & 7;
+                // Chunks from c_keep on are kept by every key of this warp: no masking.
+                const int c_keep = (r_keep + 7) >> 3;
                 for (int c = (c_warp > c_stage ? c_warp : c_stage); c < C; ++c) {
+                    const bool masked = c < c_keep;
                     uint32_t b0, b1, b2, b3;
-                    const uint32_t addr = kst + (2 * c + (mi & 1)) * 1024 + (16 * warp + 8 * (mi >> 1) + ri) * 16;
-                    ldsm_x4(addr, b0, b1, b2, b3);
-                    const int p0 = 8 * c + 2 * tq, p1 = p0 + 1;
-                    const bool ka0 = da <= (int64_t)sw[p0], ka1 = da <= (int64_t)sw[p1];
-                    const bool kb0 = db <= (int64_t)sw[p0], kb1 = db <= (int64_t)sw[p1];
-                    if (krot) {
-                        mask_pairs(b0, b1, ka0, ka1);
-                        mask_pairs(b2, b3, kb0, kb1);
-                    } else {
-                        const float th0 = sTheta[p0], th1 = sTheta[p1];
-                        const float base0 = sBase[st * H + p0], base1 = sBase[st * H + p1];
-                        float ang[4] = {fmaf(fa, th0, base0), fmaf(fa, th1, base1), fmaf(fb, th0, base0),
-                                        fmaf(fb, th1, base1)};
-                        float cs[4], sn[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const float turns = rintf(ang[u] * 0.15915494309189533577f);
-                            const float x = fmaf(-turns, 6.283185307179586477f, ang[u]);
-                            __sincosf(x, &sn[u], &cs[u]);
+                    if (kPacked) {
+                        // 64 keys x 32 B per chunk, SWIZZLE_32B; matrix mi: keys +8*(mi>>1), bytes 16*(mi&1).
+                        const int key = 16 * wq + 8 * (mi >> 1) + ri;
+                        ldsm_x4(kst + c * 2048 + key * 32 + ((16 * (mi & 1)) ^ ((key & 4) << 2)), b0, b1, b2, b3);
+                        if (masked) {
+                            const int p0 = 8 * c + tq, p1 = p0 + 4;
+                            const int w0 = sw[p0], w1 = sw[p1];
+                            b0 = (da <= w0) ? b0 : 0u;
+                            b1 = (da <= w1) ? b1 : 0u;
+                            b2 = (db <= w0) ? b2 : 0u;
+                            b3 = (db <= w1) ? b3 : 0u;
                         }
-                        rotate_pairs(b0, b1, cs[0], sn[0], cs[1], sn[1], ka0, ka1);
-                        rotate_pairs(b2, b3, cs[2], sn[2], cs[3], sn[3], kb0, kb1);
+                    } else {
+                        const uint32_t addr = kst + (2 * c + (mi & 1)) * 1024 + (16 * wq + 8 * (mi >> 1) + ri) * 16;
+                        ldsm_x4(addr, b0, b1, b2, b3);
+                        const int p0 = 8 * c + 2 * tq, p1 = p0 + 1;
+                        const int w0 = sw[p0], w1 = sw[p1];
+                        const bool ka0 = da <= w0, ka1 = da <= w1, kb0 = db <= w0, kb1 = db <= w1;
+                        if (krot) {
+                            if (masked) {
+                                mask_pairs(b0, b1, ka0, ka1);
+                                mask_pairs(b2, b3, kb0, kb1);
+                            }
+                        } else {
+                            const float th0 = sTheta[p0], th1 = sTheta[p1];
+                            const float base0 = sBase[st * H + p0], base1 = sBase[st * H + p1];
+                            float ang[4] = {fmaf(fa, th0, base0), fmaf(fa, th1, base1), fmaf(fb, th0, base0),
+                                            fmaf(fb, th1, base1)};
+                            float cs[4], sn[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const float turns = rintf(ang[u] * 0.15915494309189533577f);
+                                const float x = fmaf(-turns, 6.283185307179586477f, ang[u]);
+                                __sincosf(x, &sn[u], &cs[u]);
+                            }
+                            rotate_pairs(b0, b1, cs[0], sn[0], cs[1], sn[1], ka0, ka1);
+                            rotate_pairs(b2, b3, cs[2], sn[2], cs[3], sn[3], kb0, kb1);
+                        }
                     }
-                    mma16816(sacc[0], qa[c], b0, b1);
-                    mma16816(sacc[1], qa[c], b2, b3);
+                    // Two independent accumulation chains (chunk parity).
+                    if (c & 1) {
+                        mma16816(sodd[0], qa[c], b0, b1);
+                        mma16816(sodd[1], qa[c], b2, b3);
+                    } else {
+                        mma16816(sacc[0], qa[c], b0, b1);
+                        mma16816(sacc[1], qa[c], b2, b3);
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    sacc[0][e] += sodd[0][e];
+                    sacc[1][e] += sodd[1][e];
                 }
             }
             // Online softmax over this warp's 16 keys; rows gq (sacc[.][0..1]) and gq+8 ([2..3]).
@@ -275,8 +344,8 @@ __global__ void __launch_bounds__(kThreads) decode_tc_kernel(
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int64_t key = kw0 + 8 * nt + 2 * tq + (e & 1);
-                    const float v = (key < s1) ? sacc[nt][e] * scale_log2 : -INFINITY;
+                    const int key = kw0 + 8 * nt + 2 * tq + (e & 1);
+                    const float v = (key < (int)s1) ? sacc[nt][e] * scale_log2 : -INFINITY;
                     x[nt][e] = v;
                     tmax[e >> 1] = fmaxf(tmax[e >> 1], v);
                 }
@@ -312,23 +381,23 @@ __global__ void __launch_bounds__(kThreads) decode_tc_kernel(
             pa[1] = pack_bf16x2(p[0][2], p[0][3]);
             pa[2] = pack_bf16x2(p[1][0], p[1][1]);
             pa[3] = pack_bf16x2(p[1][2], p[1][3]);
-            if (kw0 < s1) {
+            if (kw0 < (int)s1) {
                 // O += P V: V rows = this warp's 16 keys, SW128 rows of 64 dims.
                 const uint32_t vst = sVa + st * F::VBytes;
                 const int mi = lane >> 3, ri = lane & 7;
-                const int vkey = 16 * warp + 8 * (mi & 1) + ri;
+                const int vkey = 16 * wq + 8 * (mi & 1) + ri;
 #pragma unroll
                 for (int dg = 0; dg < D / 16; ++dg) {
                     const int d0 = 16 * dg + 8 * (mi >> 1);
                     const uint32_t addr = vst + (d0 / 64) * 8192 + vkey * 128 + ((((d0 & 63) >> 3) ^ (vkey & 7)) << 4);
                     uint32_t v0, v1, v2, v3;
                     ldsm_x4_t(addr, v0, v1, v2, v3);
-                    if (kw0 + 15 >= s1) {
+                    if (kw0 + 15 >= (int)s1) {
                         // Rows past the sequence end may hold anything: P is 0 there, and
                         // 0 * (non-finite) must not reach O.  b0b1: keys 2tq, 2tq+1; b2b3: +8.
-                        const int64_t kk = kw0 + 2 * tq;
-                        const uint32_t m01 = (kk < s1 ? 0x0000FFFFu : 0u) | (kk + 1 < s1 ? 0xFFFF0000u : 0u);
-                        const uint32_t m89 = (kk + 8 < s1 ? 0x0000FFFFu : 0u) | (kk + 9 < s1 ? 0xFFFF0000u : 0u);
+                        const int kk = kw0 + 2 * tq, se = (int)s1;
+                        const uint32_t m01 = (kk < se ? 0x0000FFFFu : 0u) | (kk + 1 < se ? 0xFFFF0000u : 0u);
+                        const uint32_t m89 = (kk + 8 < se ? 0x0000FFFFu : 0u) | (kk + 9 < se ? 0xFFFF0000u : 0u);
                         v0 &= m01;
                         v1 &= m89;
                         v2 &= m01;
@@ -405,12 +474,24 @@ static cudaError_t make_map_bf16(CUtensorMap *map, const void *base, int rank, c
 }
 
 cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, const int32_t *seqlens, int krot,
-                             int nhd, const Problem &p, const WindowParams &wp, float *workspace, int split_keys,
+                             int layout, const Problem &p, const WindowParams &wp, float *workspace, int split_keys,
                              int nsplit, int *status, uint64_t limit_ns, cudaStream_t s) {
     CUtensorMap tk, tv;
     const cuuint64_t Dd = (cuuint64_t)p.D, Nm = (cuuint64_t)p.N, Hk = (cuuint64_t)p.Hkv, Bb = (cuuint64_t)p.B;
+    const int nhd = (layout == ATFLASH_KV_NHD);
+    const bool packed = (layout == ATFLASH_KV_PACKED);
     cudaError_t e;
-    if (nhd) {
+    if (packed) {
+        // K: [B*Hkv*D/16][Nmax][16] packed chunks; V: [B][Hkv][Nmax][D].
+        cuuint64_t dk[3] = {16, Nm, Bb * Hk * (Dd / 16)};
+        cuuint64_t sk[2] = {32, Nm * 32};
+        cuuint32_t boxk[3] = {16, dtc::kStageKeys, 1};
+        if ((e = make_map_bf16(&tk, kc, 3, dk, sk, boxk, CU_TENSOR_MAP_SWIZZLE_32B)) != cudaSuccess) return e;
+        cuuint64_t dims[3] = {Dd, Nm, Bb * Hk};
+        cuuint64_t str[2] = {Dd * 2, Nm * Dd * 2};
+        cuuint32_t boxv[3] = {64, dtc::kStageKeys, 1};
+        if ((e = make_map_bf16(&tv, vc, 3, dims, str, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
+    } else if (nhd) {
         cuuint64_t dims[4] = {Dd, Hk, Nm, Bb};
         cuuint64_t str[3] = {Dd * 2, Hk * Dd * 2, Nm * Hk * Dd * 2};
         cuuint32_t boxk[4] = {8, 1, dtc::kStageKeys, 1}, boxv[4] = {64, 1, dtc::kStageKeys, 1};
@@ -424,21 +505,22 @@ cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, cons
         if ((e = make_map_bf16(&tv, vc, 3, dims, str, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
     }
     dim3 grid((unsigned)nsplit, (unsigned)p.Hkv, (unsigned)p.B);
+#define ATF_DEC_TC(DD, PK)                                                                                     \
+    do {                                                                                                       \
+        const int smem = dtc::Cfg<DD>::Request;                                                                \
+        if ((e = cudaFuncSetAttribute(dtc::decode_tc_kernel<DD, PK>,                                          \
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)      \
+            return e;                                                                                          \
+        dtc::decode_tc_kernel<DD, PK><<<grid, dtc::kThreads, smem, s>>>(tk, tv, q, seqlens, workspace, p.Hq,   \
+                                                                        p.Hkv, nhd, krot, split_keys, nsplit, \
+                                                                        wp, status, limit_ns);                 \
+    } while (0)
     if (p.D == 128) {
-        const int smem = dtc::Cfg<128>::Request;
-        if ((e = cudaFuncSetAttribute(dtc::decode_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      smem)) != cudaSuccess)
-            return e;
-        dtc::decode_tc_kernel<128><<<grid, dtc::kThreads, smem, s>>>(tk, tv, q, seqlens, workspace, p.Hq, p.Hkv, nhd,
-                                                                     krot, split_keys, nsplit, wp, status, limit_ns);
+        if (packed) ATF_DEC_TC(128, true); else ATF_DEC_TC(128, false);
     } else {
-        const int smem = dtc::Cfg<64>::Request;
-        if ((e = cudaFuncSetAttribute(dtc::decode_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      smem)) != cudaSuccess)
-            return e;
-        dtc::decode_tc_kernel<64><<<grid, dtc::kThreads, smem, s>>>(tk, tv, q, seqlens, workspace, p.Hq, p.Hkv, nhd,
-                                                                    krot, split_keys, nsplit, wp, status, limit_ns);
+        if (packed) ATF_DEC_TC(64, true); else ATF_DEC_TC(64, false);
     }
+#undef ATF_DEC_TC
     return cudaGetLastError();
 }
 

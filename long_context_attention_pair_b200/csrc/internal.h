@@ -51,7 +51,7 @@ int decode_split_keys(int B, int Hkv, int64_t Nmax);
 int decode_num_splits(int B, int Hkv, int64_t Nmax);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D);
 cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, const int32_t *seqlens, int krot,
-                             int nhd, const Problem &p, const WindowParams &wp, float *workspace, int split_keys,
+                             int layout, const Problem &p, const WindowParams &wp, float *workspace, int split_keys,
                              int nsplit, int *status, uint64_t limit_ns, cudaStream_t s);
 
 // Device status word of the current device (bounded waits record timeouts
@@ -59,7 +59,7 @@ cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, cons
 int *device_status_word();
 uint64_t wait_limit_ns();
 cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const int32_t *seqlens, void *out,
-                          int out_f32, int in_f32, int krot, int nhd, const Problem &p,
+                          int out_f32, int in_f32, int krot, int layout, const Problem &p,
                           const WindowParams &wp, float *workspace, cudaStream_t s);
 
 // Driver entry point for cuTensorMapEncodeTiled (resolved once, no libcuda link).

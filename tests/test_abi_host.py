@@ -149,6 +149,8 @@ def test_decode_argument_errors(L):
     assert dec(Hq=30) == -1
     assert dec(krot=2) == -1
     assert dec(lay=5) == -1
+    assert dec(lay=atf.KV_PACKED, krot=0) == -1      # packed caches hold rotated keys
+    assert dec(lay=atf.KV_PACKED, krot=1, ind=atf.F32) == -2
     assert dec(D=80) == -2
     assert dec(Hq=68, Hkv=4) == -2   # more than 16 query heads per KV head
     assert dec(ws=None) == -3

@@ -69,6 +69,27 @@ def test_decode_matches_oracle(oracle, B, Hq, Hkv, Nmax, D, seqlens, base, kwin,
     P.check(P.host(out), ref, dtype, f"decode D={D} k={kwin} krot={krot}")
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,Nmax,D,seqlens,base,kwin", [
+    (3, 8, 2, 5000, 128, [5000, 1, 2049], 1e4, 1.0),
+    (2, 28, 4, 3000, 128, [3000, 2048], 1e7, 16.0),
+    (2, 7, 1, 4097, 64, [4097, 300], 1e6, 8.0),
+    (1, 16, 1, 900, 64, [900], 10.0, 0.25),
+])
+def test_packed_rotated_cache_matches_oracle(oracle, B, Hq, Hkv, Nmax, D, seqlens, base, kwin):
+    # The RoPE pre-pass writes the packed cache from the un-rotated keys; the oracle
+    # rotates the same un-rotated keys itself.
+    q = P.gen(23, "q_dec", (B, Hq, D), "bf16")
+    kc = P.gen(23, "k_cache", (B, Hkv, Nmax, D), "bf16")
+    vc = P.gen(23, "v_cache", (B, Hkv, Nmax, D), "bf16")
+    kpack = atf.rope_pack(kc.permute(0, 2, 1, 3).contiguous(), base)
+    sl = torch.tensor(seqlens, dtype=torch.int32, device="cuda")
+    out = atf.decode(q, kpack, vc, sl, base, kwin, kcache_rotated=True, kv_layout="PACKED",
+                     out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref = oracle.decode(P.host(q), P.host(kc), P.host(vc), seqlens, base, kwin)
+    P.check(P.host(out), ref, "bf16", f"packed decode D={D} k={kwin}")
+
+
 def test_decode_window_covering_everything_is_bit_identical_to_off():
     B, Hq, Hkv, Nmax, D, base = 2, 8, 2, 3000, 128, 1e4
     q = P.gen(22, "q_dec", (B, Hq, D), "bf16")
@@ -105,3 +126,21 @@ def test_decode_qwen7b_1m_shape(oracle, kwin):
 @pytest.mark.slow
 def test_decode_qwen7b_128k_16_seqs(oracle):
     decode_full_size(oracle, 16, 1 << 17, 16.0, seed=32)
+
+
+@pytest.mark.slow
+def test_decode_qwen7b_1m_packed_cache(oracle):
+    B, L, Hq, Hkv, D, base, kwin = 4, 1 << 20, 28, 4, 128, 1e7, 16.0
+    q = P.gen(33, "q_dec", (B, Hq, D), "bf16")
+    kc = P.gen(33, "k_cache", (B, Hkv, L, D), "bf16")
+    vc = P.gen(33, "v_cache", (B, Hkv, L, D), "bf16")
+    kpack = atf.rope_pack(kc.permute(0, 2, 1, 3).contiguous(), base)
+    sl = torch.full((B,), L, dtype=torch.int32, device="cuda")
+    out = atf.decode(q, kpack, vc, sl, base, kwin, kcache_rotated=True, kv_layout="PACKED",
+                     out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    got = P.host(out)
+    del kpack
+    for b in range(B):
+        ref = oracle.decode(P.host(q[b:b + 1]), P.host(kc[b:b + 1]), P.host(vc[b:b + 1]), [L], base, kwin)
+        P.check(got[b:b + 1], ref, "bf16", f"packed decode 1M b={b}")
