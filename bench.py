@@ -231,7 +231,7 @@ def cpu_baseline(q, k, v, wl, budget_s=12.0):
         return time.perf_counter() - t0
 
     t = run(8)
-    nrows = int(max(8, min(1024, 8 * budget_s / max(t, 1e-3))))
+    nrows = int(max(8, min(N, 8 * budget_s / max(t, 1e-3))))
     t = run(nrows)
     return {"value": nrows / t, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
             "sample": f"{nrows} uniformly drawn query rows x all {wl['Hq']} heads of the workload "
