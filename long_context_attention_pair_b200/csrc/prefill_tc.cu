@@ -23,15 +23,14 @@
 // softmax warpgroups ping-pong with the tensor core.  12 warps:
 //   warps 0-3 / 4-7  softmax of head 0 / head 1: one TMEM lane quarter each;
 //                    boundary fix-up, causal mask, online softmax in the log2
-//                    domain, P (bf16) written back over S in TMEM, O rescale
-//                    (only when the running max grows by more than 2^8),
-//                    epilogue O / l
+//                    domain, P (bf16) into TMEM, O rescale (only when the
+//                    running max grows by more than 2^8), epilogue O / l
 //   warp 8           TMA producer (Q~ once; K~ chunks and V per key tile)
 //   warp 9           TMEM owner and MMA issuer: S_h = Q~_h K~^T (smem x smem),
 //                    O_h += P_h V (P from TMEM, V from smem)
 //   warp 10          zeroes the fully-pruned pairs of the first loaded K~ chunk
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D);
-// P_h occupies the first 64 columns of S_h once S_h has been read.
+//                    and stages the tile's boundary pairs as fp32 for the fix-up
+// TMEM columns: O0 [256,256+D), O1 [256+D,256+2D); S and P as in Cfg below.
 // Every mbarrier wait is bounded in time; on expiry the CTA records
 // ATFLASH_ERR_TIMEOUT in the device status word, lets its copies land, drains
 // its tensor-core work, frees TMEM and exits.
@@ -78,9 +77,13 @@ struct Cfg {
     static constexpr int Total = OffCtl + 2048;
     static constexpr int Request = Total + 1024;
     static constexpr uint32_t TmemO0 = 256, TmemO1 = 256 + D;
-    // D = 64 leaves 128 TMEM columns for P of its own; D = 128 writes P over S.
-    static constexpr bool SepP = (D == 64);
-    static constexpr uint32_t TmemP0 = SepP ? 384 : 0, TmemP1 = SepP ? 448 : 128;
+    // TMEM: D = 64: S0 [0,128), S1 [128,256), O0, O1 [256,384), P0, P1 [384,512).
+    //       D = 128: one S [0,128) shared by the two heads in turn, P0 [128,192),
+    //                P1 [192,256), O0 [256,384), O1 [384,512).
+    // Either way S_t is free again as soon as softmax t has read it into registers.
+    static constexpr bool SharedS = (D == 128);
+    static constexpr uint32_t TmemS0 = 0, TmemS1 = SharedS ? 0 : 128;
+    static constexpr uint32_t TmemP0 = SharedS ? 128 : 384, TmemP1 = SharedS ? 192 : 448;
 };
 
 template <int KS, int VS>
@@ -318,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = ca; c < C; ++c) {
                     const uint64_t da = smem_desc(sQa + t * F::QBytes + c * kChunkBytes, 16, 256, kSwizzle32B);
                     const uint64_t db = smem_desc(sKa + ks * F::KBytes + c * kChunkBytes, 16, 256, kSwizzle32B);
-                    umma_bf16_ss(tmem + t * 128, da, db, idesc_qk, c > ca ? 1u : 0u);
+                    umma_bf16_ss(tmem + (t ? F::TmemS1 : F::TmemS0), da, db, idesc_qk, c > ca ? 1u : 0u);
                 }
                 umma_commit(&ctl->s_full[t]);
             }
@@ -355,10 +358,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             wc.site = 7;
             if (!(ok = mbar_wait_warp(&ctl->k_ready[ks], (j / KS) & 1, wc))) break;
             if (lane == 0) tc_fence_after();
-            if constexpr (F::SepP) {
+            wc.site = 13;
+            if constexpr (F::SharedS) {
+                // One S for both heads: S_0(j) once head 1 has read S_1(j-1), S_1(j) once
+                // head 0 has read S_0(j).  PV_0(j-1) goes in between (its P_0 is ready
+                // before softmax 0 reads S_0(j)).
+                if (j > 0) {
+                    uint64_t *free_bar = two ? &ctl->s_read[1] : &ctl->s_read[0];
+                    if (!(ok = mbar_wait_warp(free_bar, (j - 1) & 1, wc))) break;
+                }
+                if (lane == 0) tc_fence_after();
+                issue_qk(0, ks, ca);
+                if (j > 0 && !(ok = issue_pv(0, j - 1, !two))) break;
+                if (two) {
+                    if (!(ok = mbar_wait_warp(&ctl->s_read[0], j & 1, wc))) break;
+                    if (lane == 0) tc_fence_after();
+                    issue_qk(1, ks, ca);
+                }
+                if (lane == 0) umma_commit(&ctl->k_empty[ks]);
+                __syncwarp();
+                if (two && j > 0 && !(ok = issue_pv(1, j - 1, true))) break;
+            } else {
                 // S_t(j) as soon as softmax t has read S_t(j-1); PV of the previous
                 // tile follows once its P is written.
-                wc.site = 13;
                 if (j > 0 && !(ok = mbar_wait_warp(&ctl->s_read[0], (j - 1) & 1, wc))) break;
                 if (lane == 0) tc_fence_after();
                 issue_qk(0, ks, ca);
@@ -373,19 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!(ok = issue_pv(0, j - 1, !two))) break;
                     if (two && !(ok = issue_pv(1, j - 1, true))) break;
                 }
-            } else {
-                // P_t is written over S_t: S_t(j) only after PV_t(j-1) was issued.
-                issue_qk(0, ks, ca);
-                if (two && j > 0 && !(ok = issue_pv(1, j - 1, true))) break;
-                if (two) issue_qk(1, ks, ca);
-                if (lane == 0) umma_commit(&ctl->k_empty[ks]);
-                __syncwarp();
-                if (!(ok = issue_pv(0, j, !two))) break;
             }
         }
-        if constexpr (F::SepP) {
-            if (ok) ok = issue_pv(0, nkt - 1, !two);
-        }
+        if (ok) ok = issue_pv(0, nkt - 1, !two);
         if (ok && two) ok = issue_pv(1, nkt - 1, true);
     } else if (warp < 8) {
         // ------------------------------------------------------------- softmax
@@ -397,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int64_t n = n0 + row;
             const int hq = h0 + t;
             const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-            const uint32_t tS = tmem + (uint32_t)(t * 128) + lane_off;
+            const uint32_t tS = tmem + (t ? F::TmemS1 : F::TmemS0) + lane_off;
             const uint32_t tP = tmem + (t ? F::TmemP1 : F::TmemP0) + lane_off;
             const uint32_t tO = tmem + (t ? F::TmemO1 : F::TmemO0) + lane_off;
             const uint8_t *sQt = sQ + t * F::QBytes;
@@ -436,12 +448,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < kBN; ++i) s[i] = 0.f;
                 }
-                if constexpr (F::SepP) {
-                    // S_t(j) is in registers: the MMA may overwrite it with S_t(j+1).
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&ctl->s_read[t]);
-                }
+                // S is in registers: the MMA may reuse its columns.
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->s_read[t]);
                 // Boundary pairs: the dense MMA included them; remove them from the
                 // cells whose distance exceeds the pair's window (jj < n - m0 - w_r).
                 if (bd.r_lo < bd.r_full) {
@@ -557,9 +567,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pk[i + 1] = pack_bf16x2(xb.x, xb.y);
                 }
                 // Rescale O only when some row's max grew past the threshold (rare).
-                // With P in its own columns, PV_t(j-1) must also be done reading P.
+                // PV_t(j-1) must also be done reading P_t before it is overwritten.
                 const bool rescale = (j > 0) && __any_sync(0xffffffffu, need);
-                if (j > 0 && (F::SepP || rescale)) {
+                if (j > 0) {
                     wc.site = 11;
                     if (!(ok = mbar_wait_warp(&ctl->o_done[t], (j - 1) & 1, wc))) break;
                     tc_fence_after();
@@ -575,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_st_32x32b_x32(tO + cc * 32, r);
                     }
                 }
-                // P (its own columns, or the first 64 columns of S, read in full above).
+                // P_t (bf16 pairs) into its own 64 columns.
                 {
                     uint32_t (&pa)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
                     uint32_t (&pb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
