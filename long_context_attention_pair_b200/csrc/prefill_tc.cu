@@ -26,10 +26,10 @@
 //                    domain, P (bf16) into TMEM, O rescale (only when the
 //                    running max grows by more than 2^8), epilogue O / l
 //   warp 8           TMA producer (Q~ once; K~ chunks and V per key tile)
-//   warp 9           TMEM owner and MMA issuer: S_h = Q~_h K~^T (smem x smem),
-//                    O_h += P_h V (P from TMEM, V from smem)
+//   warp 9           TMEM owner and QK issuer: S_h = Q~_h K~^T (smem x smem)
 //   warp 10          zeroes the fully-pruned pairs of the first loaded K~ chunk
 //                    and stages the tile's boundary pairs as fp32 for the fix-up
+//   warp 11          PV issuer: O_h += P_h V (P from TMEM, V from smem)
 // TMEM columns: O0 [256,256+D), O1 [256+D,256+2D); S and P as in Cfg below.
 // Every mbarrier wait is bounded in time; on expiry the CTA records
 // ATFLASH_ERR_TIMEOUT in the device status word, lets its copies land, drains
@@ -47,7 +47,7 @@ namespace tc {
 constexpr int kBM = 128;
 constexpr int kBN = 128;
 constexpr int kThreads = 384;
-constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpFix = 10;
+constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpFix = 10, kWarpPv = 11;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kChunkBytes = kBN * 32;  // 128 rows x 16 bf16 (one K-step)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
@@ -82,6 +82,7 @@ struct Cfg {
     //                P1 [192,256), O0 [256,384), O1 [384,512).
     // Either way S_t is free again as soon as softmax t has read it into registers.
     static constexpr bool SharedS = (D == 128);
+    static constexpr bool Token = false;  // alternate the two heads' exp2 passes (measured slower)
     static constexpr uint32_t TmemS0 = 0, TmemS1 = SharedS ? 0 : 128;
     static constexpr uint32_t TmemP0 = SharedS ? 128 : 384, TmemP1 = SharedS ? 192 : 448;
 };
@@ -93,6 +94,7 @@ struct Ctl {
     uint64_t v_full[VS], v_empty[VS];
     uint64_t s_full[2], s_read[2], p_full[2], o_done[2];
     uint64_t drain;
+    uint64_t tok[2][4];  // [head][warp of the head]: that warp finished its exp2 pass of a tile
     uint32_t tmem_base;
     int abort_flag;
     int w[kMaxPairs];
@@ -207,7 +209,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&ctl->p_full[s], 4);
             mbar_init(&ctl->o_done[s], 1);
         }
-        mbar_init(&ctl->drain, 1);
+        mbar_init(&ctl->drain, 2);  // one commit from each issuing warp
+        for (int t = 0; t < 2; ++t)
+            for (int q = 0; q < 4; ++q) mbar_init(&ctl->tok[t][q], 1);
         ctl->abort_flag = 0;
         fence_mbar_init();
     }
@@ -310,14 +314,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&ctl->k_ready[ks]);
         }
     } else if (warp == kWarpMma) {
-        // ---------------------------------------------------------- MMA issuer
+        // ------------------------------------------------------- QK issuer
+        // tcgen05.mma issue returns only once the tensor pipe has taken the
+        // instruction, so a warp that issued PV could not start the next QK
+        // early; QK and PV therefore have an issuing warp each.
         const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
-        const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
-        const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+        const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
         wc.site = 4;
         bool ok = mbar_wait_warp(&ctl->q_full, 0, wc);
         auto issue_qk = [&](int t, int ks, int ca) {
             if (lane == 0) {
+                tc_fence_after();
                 for (int c = ca; c < C; ++c) {
                     const uint64_t da = smem_desc(sQa + t * F::QBytes + c * kChunkBytes, 16, 256, kSwizzle32B);
                     const uint64_t db = smem_desc(sKa + ks * F::KBytes + c * kChunkBytes, 16, 256, kSwizzle32B);
@@ -327,29 +334,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
         };
-        auto issue_pv = [&](int t, int jj, bool release_v) -> bool {
-            const int vs = jj % VS;
-            wc.site = 5;
-            if (!mbar_wait_warp(&ctl->v_full[vs], (jj / VS) & 1, wc)) return false;
-            wc.site = 6;
-            if (!mbar_wait_warp(&ctl->p_full[t], jj & 1, wc)) return false;
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t o_col = t ? F::TmemO1 : F::TmemO0;
-#pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    // A = P_t keys [16kk, 16kk+16): 8 TMEM columns of bf16 pairs.
-                    // B = V rows [16kk, 16kk+16): MN-major SW128, 64-dim groups 16 KB apart.
-                    const uint64_t db = smem_desc(sVa + vs * F::VBytes + kk * 2048, 16384, 1024, kSwizzle128B);
-                    umma_bf16_ts(tmem + o_col, tmem + (t ? F::TmemP1 : F::TmemP0) + kk * 8, db, idesc_pv,
-                                 (jj > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(&ctl->o_done[t]);
-                if (release_v) umma_commit(&ctl->v_empty[vs]);
-            }
-            __syncwarp();
-            return true;
-        };
         BandWalk bw;
         bw.init(w, H, n0);
         for (int j = 0; j < nkt && ok; ++j) {
@@ -357,48 +341,55 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ca = bw.at(w, n0, (int64_t)j * kBN).r_lo >> 3;
             wc.site = 7;
             if (!(ok = mbar_wait_warp(&ctl->k_ready[ks], (j / KS) & 1, wc))) break;
-            if (lane == 0) tc_fence_after();
+            // S_0(j) once its columns are free: read by head 0 (own buffer) or by
+            // head 1 (buffer shared by the two heads); S_1(j) likewise.
             wc.site = 13;
-            if constexpr (F::SharedS) {
-                // One S for both heads: S_0(j) once head 1 has read S_1(j-1), S_1(j) once
-                // head 0 has read S_0(j).  PV_0(j-1) goes in between (its P_0 is ready
-                // before softmax 0 reads S_0(j)).
-                if (j > 0) {
-                    uint64_t *free_bar = two ? &ctl->s_read[1] : &ctl->s_read[0];
-                    if (!(ok = mbar_wait_warp(free_bar, (j - 1) & 1, wc))) break;
-                }
-                if (lane == 0) tc_fence_after();
-                issue_qk(0, ks, ca);
-                if (j > 0 && !(ok = issue_pv(0, j - 1, !two))) break;
-                if (two) {
-                    if (!(ok = mbar_wait_warp(&ctl->s_read[0], j & 1, wc))) break;
-                    if (lane == 0) tc_fence_after();
-                    issue_qk(1, ks, ca);
-                }
-                if (lane == 0) umma_commit(&ctl->k_empty[ks]);
-                __syncwarp();
-                if (two && j > 0 && !(ok = issue_pv(1, j - 1, true))) break;
-            } else {
-                // S_t(j) as soon as softmax t has read S_t(j-1); PV of the previous
-                // tile follows once its P is written.
-                if (j > 0 && !(ok = mbar_wait_warp(&ctl->s_read[0], (j - 1) & 1, wc))) break;
-                if (lane == 0) tc_fence_after();
-                issue_qk(0, ks, ca);
-                if (two) {
-                    if (j > 0 && !(ok = mbar_wait_warp(&ctl->s_read[1], (j - 1) & 1, wc))) break;
-                    if (lane == 0) tc_fence_after();
-                    issue_qk(1, ks, ca);
-                }
-                if (lane == 0) umma_commit(&ctl->k_empty[ks]);
-                __syncwarp();
-                if (j > 0) {
-                    if (!(ok = issue_pv(0, j - 1, !two))) break;
-                    if (two && !(ok = issue_pv(1, j - 1, true))) break;
-                }
+            if (j > 0) {
+                uint64_t *free_bar = (F::SharedS && two) ? &ctl->s_read[1] : &ctl->s_read[0];
+                if (!(ok = mbar_wait_warp(free_bar, (j - 1) & 1, wc))) break;
             }
+            issue_qk(0, ks, ca);
+            if (two) {
+                if (F::SharedS) {
+                    if (!(ok = mbar_wait_warp(&ctl->s_read[0], j & 1, wc))) break;
+                } else if (j > 0) {
+                    if (!(ok = mbar_wait_warp(&ctl->s_read[1], (j - 1) & 1, wc))) break;
+                }
+                issue_qk(1, ks, ca);
+            }
+            if (lane == 0) umma_commit(&ctl->k_empty[ks]);
+            __syncwarp();
         }
-        if (ok) ok = issue_pv(0, nkt - 1, !two);
-        if (ok && two) ok = issue_pv(1, nkt - 1, true);
+    } else if (warp == kWarpPv) {
+        // ------------------------------------------------------- PV issuer
+        const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
+        const uint32_t sVa = smem_u32(sV);
+        bool ok = true;
+        for (int j = 0; j < nkt && ok; ++j) {
+            const int vs = j % VS;
+            wc.site = 5;
+            if (!(ok = mbar_wait_warp(&ctl->v_full[vs], (j / VS) & 1, wc))) break;
+            for (int t = 0; t < nwg && ok; ++t) {
+                wc.site = 6;
+                if (!(ok = mbar_wait_warp(&ctl->p_full[t], j & 1, wc))) break;
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t o_col = t ? F::TmemO1 : F::TmemO0;
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk) {
+                        // A = P_t keys [16kk, 16kk+16): 8 TMEM columns of bf16 pairs.
+                        // B = V rows [16kk, 16kk+16): MN-major SW128, 64-dim groups 16 KB apart.
+                        const uint64_t db = smem_desc(sVa + vs * F::VBytes + kk * 2048, 16384, 1024, kSwizzle128B);
+                        umma_bf16_ts(tmem + o_col, tmem + (t ? F::TmemP1 : F::TmemP0) + kk * 8, db, idesc_pv,
+                                     (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&ctl->o_done[t]);
+                }
+                __syncwarp();
+            }
+            if (ok && lane == 0) umma_commit(&ctl->v_empty[vs]);
+            __syncwarp();
+        }
     } else if (warp < 8) {
         // ------------------------------------------------------------- softmax
         setmaxnreg_inc<200>();
@@ -540,6 +531,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float m_new = need ? tile_max : m_used;
                 const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
                 m_used = m_new;
+                // The two heads' warps on one SM sub-partition take turns at the exp2
+                // pass (head 0 of tile j, head 1 of tile j, head 0 of tile j+1, ...), so
+                // that the multi-function unit serves one of them at a time while the
+                // other loads S, corrects it and stores P.
+                if (F::Token && two) {
+                    wc.site = 14;
+                    if (t == 1) ok = mbar_wait_warp(&ctl->tok[0][q4], j & 1, wc);
+                    else if (j > 0) ok = mbar_wait_warp(&ctl->tok[1][q4], (j - 1) & 1, wc);
+                    if (!ok) break;
+                }
                 // P = exp2(s * scale - m) as bf16 pairs; S registers die as P is produced.
                 const float2 mneg = make_float2(-m_used, -m_used);
                 const float2 sc2 = make_float2(scale_log2, scale_log2);
@@ -565,6 +566,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     l1 = add2(l1, xb);
                     pk[i] = pack_bf16x2(xa.x, xa.y);
                     pk[i + 1] = pack_bf16x2(xb.x, xb.y);
+                }
+                if (F::Token && two) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ctl->tok[t][q4]);
                 }
                 // Rescale O only when some row's max grew past the threshold (rare).
                 // PV_t(j-1) must also be done reading P_t before it is overwritten.
@@ -646,6 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // Teardown: every tensor-core operation must be complete before TMEM is freed.
     __syncthreads();
+    if (warp == kWarpPv && lane == 0) umma_commit(&ctl->drain);
     if (warp == kWarpMma) {
         if (lane == 0) {
             umma_commit(&ctl->drain);
