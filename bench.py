@@ -526,6 +526,8 @@ def main():
         raise SystemExit("need --steps >= 1 and --warmup >= 3")
     if args.workload in DECODE_WORKLOADS:
         wl = dict(DECODE_WORKLOADS[args.workload])
+        if args.N:
+            wl["N"] = args.N
         if args.k_window is not None:
             wl["k_window"] = args.k_window
         run_decode(args, wl)
