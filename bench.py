@@ -83,7 +83,7 @@ KERNELS_PER_STEP = 5  # rope_pack(q), rope_pack(k), prefill_tc, decode_split, de
 # DRAM bytes per launch of the tcgen05 prefill kernel on this workload, from one
 # ncu capture (profiles/prefill_tc_qwen05b_32k.md).  Valid only while the
 # kernel source hashes to `source_sha1`; otherwise the line reports null.
-TRAFFIC = {"bytes_per_launch": None, "source_sha1": None}
+TRAFFIC = {"bytes_per_launch": 98930944, "source_sha1": "d7bb473dfa1cc9a4b88a7ba8fb42edfb2750ff10"}
 
 
 def parse():
@@ -173,7 +173,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self._gpu_id(), "--query-gpu=" + ",".join(self.FIELDS),
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -454,6 +454,7 @@ def run_decode(args, wl):
 
     sampler = ClockSampler(local)
     sampler.start()
+    time.sleep(0.3)
     ms = timed(kwin, args.steps)
     clocks = sampler.stop()
     ms_off = timed(math.inf, args.steps)
