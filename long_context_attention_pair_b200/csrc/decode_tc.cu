@@ -278,15 +278,26 @@ __global__ void __launch_bounds__(kThreads) decode_tc_kernel(
                 const float fa = (float)(16 * wq + gq), fb = fa + 8.f;
                 const uint32_t kst = sKa + st * F::KBytes;
                 const int mi = lane >> 3, ri = lane & 7;
-                // Chunks from c_keep on are kept by every key of this warp: no masking.
                 const int c_keep = (r_keep + 7) >> 3;
-                for (int c = (c_warp > c_stage ? c_warp : c_stage); c < C; ++c) {
-                    const bool masked = c < c_keep;
-                    uint32_t b0, b1, b2, b3;
-                    if (kPacked) {
+                if constexpr (kPacked) {
+                    const int c_begin = c_warp > c_stage ? c_warp : c_stage;
+                    // All of this warp's K fragments first (independent shared-memory loads in
+                    // flight together), then the masks and the MMAs.
+                    uint32_t kb[C][4];
+#pragma unroll
+                    for (int c = 0; c < C; ++c) {
+                        if (c < c_begin) continue;
                         // 64 keys x 32 B per chunk, SWIZZLE_32B; matrix mi: keys +8*(mi>>1), bytes 16*(mi&1).
                         const int key = 16 * wq + 8 * (mi >> 1) + ri;
-                        ldsm_x4(kst + c * 2048 + key * 32 + ((16 * (mi & 1)) ^ ((key & 4) << 2)), b0, b1, b2, b3);
+                        ldsm_x4(kst + c * 2048 + key * 32 + ((16 * (mi & 1)) ^ ((key & 4) << 2)), kb[c][0], kb[c][1],
+                                kb[c][2], kb[c][3]);
+                    }
+#pragma unroll
+                    for (int c = 0; c < C; ++c) {
+                        if (c < c_begin) continue;
+                        // Chunks from c_keep on are kept by every key of this warp: no masking.
+                        const bool masked = c < c_keep;
+                        uint32_t b0 = kb[c][0], b1 = kb[c][1], b2 = kb[c][2], b3 = kb[c][3];
                         if (masked) {
                             const int p0 = 8 * c + tq, p1 = p0 + 4;
                             const int w0 = sw[p0], w1 = sw[p1];
@@ -295,40 +306,66 @@ __global__ void __launch_bounds__(kThreads) decode_tc_kernel(
                             b2 = (db <= w0) ? b2 : 0u;
                             b3 = (db <= w1) ? b3 : 0u;
                         }
-                    } else {
-                        const uint32_t addr = kst + (2 * c + (mi & 1)) * 1024 + (16 * wq + 8 * (mi >> 1) + ri) * 16;
-                        ldsm_x4(addr, b0, b1, b2, b3);
-                        const int p0 = 8 * c + 2 * tq, p1 = p0 + 1;
-                        const int w0 = sw[p0], w1 = sw[p1];
-                        const bool ka0 = da <= w0, ka1 = da <= w1, kb0 = db <= w0, kb1 = db <= w1;
-                        if (krot) {
-                            if (masked) {
-                                mask_pairs(b0, b1, ka0, ka1);
-                                mask_pairs(b2, b3, kb0, kb1);
-                            }
+                        // Two independent accumulation chains (chunk parity).
+                        if (c & 1) {
+                            mma16816(sodd[0], qa[c], b0, b1);
+                            mma16816(sodd[1], qa[c], b2, b3);
                         } else {
-                            const float th0 = sTheta[p0], th1 = sTheta[p1];
-                            const float base0 = sBase[st * H + p0], base1 = sBase[st * H + p1];
-                            float ang[4] = {fmaf(fa, th0, base0), fmaf(fa, th1, base1), fmaf(fb, th0, base0),
-                                            fmaf(fb, th1, base1)};
-                            float cs[4], sn[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const float turns = rintf(ang[u] * 0.15915494309189533577f);
-                                const float x = fmaf(-turns, 6.283185307179586477f, ang[u]);
-                                __sincosf(x, &sn[u], &cs[u]);
-                            }
-                            rotate_pairs(b0, b1, cs[0], sn[0], cs[1], sn[1], ka0, ka1);
-                            rotate_pairs(b2, b3, cs[2], sn[2], cs[3], sn[3], kb0, kb1);
+                            mma16816(sacc[0], qa[c], b0, b1);
+                            mma16816(sacc[1], qa[c], b2, b3);
                         }
                     }
-                    // Two independent accumulation chains (chunk parity).
-                    if (c & 1) {
-                        mma16816(sodd[0], qa[c], b0, b1);
-                        mma16816(sodd[1], qa[c], b2, b3);
-                    } else {
-                        mma16816(sacc[0], qa[c], b0, b1);
-                        mma16816(sacc[1], qa[c], b2, b3);
+                } else {
+                    for (int c = (c_warp > c_stage ? c_warp : c_stage); c < C; ++c) {
+                        const bool masked = c < c_keep;
+                        uint32_t b0, b1, b2, b3;
+                        if (kPacked) {
+                            // 64 keys x 32 B per chunk, SWIZZLE_32B; matrix mi: keys +8*(mi>>1), bytes 16*(mi&1).
+                            const int key = 16 * wq + 8 * (mi >> 1) + ri;
+                            ldsm_x4(kst + c * 2048 + key * 32 + ((16 * (mi & 1)) ^ ((key & 4) << 2)), b0, b1, b2, b3);
+                            if (masked) {
+                                const int p0 = 8 * c + tq, p1 = p0 + 4;
+                                const int w0 = sw[p0], w1 = sw[p1];
+                                b0 = (da <= w0) ? b0 : 0u;
+                                b1 = (da <= w1) ? b1 : 0u;
+                                b2 = (db <= w0) ? b2 : 0u;
+                                b3 = (db <= w1) ? b3 : 0u;
+                            }
+                        } else {
+                            const uint32_t addr = kst + (2 * c + (mi & 1)) * 1024 + (16 * wq + 8 * (mi >> 1) + ri) * 16;
+                            ldsm_x4(addr, b0, b1, b2, b3);
+                            const int p0 = 8 * c + 2 * tq, p1 = p0 + 1;
+                            const int w0 = sw[p0], w1 = sw[p1];
+                            const bool ka0 = da <= w0, ka1 = da <= w1, kb0 = db <= w0, kb1 = db <= w1;
+                            if (krot) {
+                                if (masked) {
+                                    mask_pairs(b0, b1, ka0, ka1);
+                                    mask_pairs(b2, b3, kb0, kb1);
+                                }
+                            } else {
+                                const float th0 = sTheta[p0], th1 = sTheta[p1];
+                                const float base0 = sBase[st * H + p0], base1 = sBase[st * H + p1];
+                                float ang[4] = {fmaf(fa, th0, base0), fmaf(fa, th1, base1), fmaf(fb, th0, base0),
+                                                fmaf(fb, th1, base1)};
+                                float cs[4], sn[4];
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    const float turns = rintf(ang[u] * 0.15915494309189533577f);
+                                    const float x = fmaf(-turns, 6.283185307179586477f, ang[u]);
+                                    __sincosf(x, &sn[u], &cs[u]);
+                                }
+                                rotate_pairs(b0, b1, cs[0], sn[0], cs[1], sn[1], ka0, ka1);
+                                rotate_pairs(b2, b3, cs[2], sn[2], cs[3], sn[3], kb0, kb1);
+                            }
+                        }
+                        // Two independent accumulation chains (chunk parity).
+                        if (c & 1) {
+                            mma16816(sodd[0], qa[c], b0, b1);
+                            mma16816(sodd[1], qa[c], b2, b3);
+                        } else {
+                            mma16816(sacc[0], qa[c], b0, b1);
+                            mma16816(sacc[1], qa[c], b2, b3);
+                        }
                     }
                 }
 #pragma unroll
