@@ -113,8 +113,11 @@ __device__ __forceinline__ void mask_pairs(uint32_t &lo, uint32_t &hi, bool keep
     hi &= m;
 }
 
+// The natural-layout kernel (rotation at load) is asked for two CTAs per SM, which
+// lets the compiler use more registers than its default; the packed kernel keeps
+// the default, which measured faster.
 template <int D, bool kPacked>
-__global__ void __launch_bounds__(kThreads) decode_tc_kernel(
+__global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const void *q_,
     const int32_t *__restrict__ seqlens, float *__restrict__ ws, int Hq, int Hkv, int nhd, int krot, int split_keys,
     int nsplit, const __grid_constant__ WindowParams wp, int *status, uint64_t limit_ns) {
