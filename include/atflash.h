@@ -210,6 +210,27 @@ int atflash_decode_noalloc(const void *q, const void *kcache, const void *vcache
  */
 int atflash_device_status(int clear);
 
+/*
+ * Limit, in milliseconds, of every pipeline wait (an mbarrier wait between the
+ * warps of a CTA) in the kernels launched after this call; initially
+ * ATFLASH_WAIT_LIMIT_MS from the environment, else 2000.  When a wait runs out
+ * the CTA records ATFLASH_ERR_TIMEOUT in the device status word, lets its own
+ * copies and tensor-core work finish (those waits use at least 200 ms) and
+ * exits; its output is then incomplete.  Returns ATFLASH_ERR_INVALID_ARG unless
+ * 0 < ms <= 60000.  Not part of the method; it exists to bound failures.
+ */
+int atflash_set_wait_limit_ms(double ms);
+
+/*
+ * Failure-detection self-test: launches one CTA on `stream` that waits, with
+ * the bounded wait the kernels use, on an mbarrier that nothing completes, for
+ * `limit_ms` milliseconds (0 < limit_ms <= 10000), then records
+ * ATFLASH_ERR_TIMEOUT in the device status word and returns.  The call itself
+ * returns ATFLASH_OK once launched; read the outcome with
+ * atflash_device_status.  Not part of the method.
+ */
+int atflash_selftest_wait_timeout(double limit_ms, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

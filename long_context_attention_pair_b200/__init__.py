@@ -257,3 +257,21 @@ def decode(q, k_cache, v_cache, seqlens, rope_base: float, k_window: float = mat
 def device_status(clear: bool = True) -> int:
     """ATFlash device status word (0, or -5 after a kernel's bounded wait ran out)."""
     return int(lib().atflash_device_status(1 if clear else 0))
+
+
+def set_wait_limit_ms(ms: float) -> None:
+    """Limit of the kernels' pipeline waits for launches after this call."""
+    f = lib().atflash_set_wait_limit_ms
+    f.argtypes = [ctypes.c_double]
+    f.restype = ctypes.c_int
+    _check(f(float(ms)), "atflash_set_wait_limit_ms")
+
+
+def selftest_wait_timeout(limit_ms: float, stream=None) -> None:
+    """Launch the failure-detection self-test (a bounded wait that must run out)."""
+    import torch
+    f = lib().atflash_selftest_wait_timeout
+    f.argtypes = [ctypes.c_double, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    st = (stream or torch.cuda.current_stream()).cuda_stream
+    _check(f(float(limit_ms), ctypes.c_void_p(st)), "atflash_selftest_wait_timeout")

@@ -7,6 +7,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -67,16 +68,21 @@ EncodeTiledFn encode_tiled_fn() {
     return fn;
 }
 
+// Limit of every pipeline wait in the kernels: ATFLASH_WAIT_LIMIT_MS at first
+// use (default 2000 ms), changed by atflash_set_wait_limit_ms.
+static std::atomic<uint64_t> g_wait_limit_ns{0};
+
 uint64_t wait_limit_ns() {
-    static uint64_t v = 0;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        const char *e = getenv("ATFLASH_WAIT_LIMIT_MS");
-        double ms = e ? atof(e) : 2000.0;
-        if (!(ms > 0)) ms = 2000.0;
-        v = (uint64_t)(ms * 1e6);
-    });
-    return v;
+    uint64_t v = g_wait_limit_ns.load();
+    if (v) return v;
+    const char *e = getenv("ATFLASH_WAIT_LIMIT_MS");
+    double ms = e ? atof(e) : 2000.0;
+    if (!(ms > 0)) ms = 2000.0;
+    uint64_t want = (uint64_t)(ms * 1e6);
+    if (want == 0) want = 1;
+    uint64_t expected = 0;
+    g_wait_limit_ns.compare_exchange_strong(expected, want);
+    return g_wait_limit_ns.load();
 }
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -306,6 +312,23 @@ int atflash_device_status(int clear) {
         if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(int)) != cudaSuccess) return ATFLASH_ERR_CUDA;
     }
     return v >= ATFLASH_DEVICE_TIMEOUT_BASE ? ATFLASH_ERR_TIMEOUT : ATFLASH_OK;
+}
+
+int atflash_set_wait_limit_ms(double ms) {
+    if (!(ms > 0.0) || ms > 60000.0) return ATFLASH_ERR_INVALID_ARG;
+    uint64_t v = (uint64_t)(ms * 1e6);
+    if (v == 0) v = 1;
+    g_wait_limit_ns.store(v);
+    return ATFLASH_OK;
+}
+
+int atflash_selftest_wait_timeout(double limit_ms, cudaStream_t stream) {
+    if (!(limit_ms > 0.0) || limit_ms > 10000.0) return ATFLASH_ERR_INVALID_ARG;
+    int *status = device_status_word();
+    if (!status) return ATFLASH_ERR_CUDA;
+    uint64_t v = (uint64_t)(limit_ms * 1e6);
+    if (v == 0) v = 1;
+    return launch_selftest_wait(status, v, stream) == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
                 if (last[s] < 0) continue;
                 const uint64_t t0 = globaltimer_ns();
                 while (!mbar_try_wait(&bars->full[s], (last[s] / kStages) & 1))
-                    if (globaltimer_ns() - t0 > limit_ns) break;
+                    if (globaltimer_ns() - t0 > atflash_drain_limit_ns(limit_ns)) break;
             }
         }
     } else {

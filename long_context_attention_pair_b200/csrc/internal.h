@@ -58,6 +58,8 @@ cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, cons
 // here) and the wait limit in nanoseconds.
 int *device_status_word();
 uint64_t wait_limit_ns();
+// One CTA whose bounded wait on an mbarrier that nothing completes runs out.
+cudaError_t launch_selftest_wait(int *status, uint64_t limit_ns, cudaStream_t s);
 cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const int32_t *seqlens, void *out,
                           int out_f32, int in_f32, int krot, int layout, const Problem &p,
                           const WindowParams &wp, float *workspace, cudaStream_t s);

@@ -269,11 +269,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) {
                 // Let every copy this thread started land before the CTA exits.
-                wait_drain(&ctl->q_full, 0, limit_ns);
+                const uint64_t drain_ns = atflash_drain_limit_ns(limit_ns);
+                wait_drain(&ctl->q_full, 0, drain_ns);
                 for (int s = 0; s < KS; ++s)
-                    if (last_k[s] >= 0) wait_drain(&ctl->k_full[s], (last_k[s] / KS) & 1, limit_ns);
+                    if (last_k[s] >= 0) wait_drain(&ctl->k_full[s], (last_k[s] / KS) & 1, drain_ns);
                 for (int s = 0; s < VS; ++s)
-                    if (last_v[s] >= 0) wait_drain(&ctl->v_full[s], (last_v[s] / VS) & 1, limit_ns);
+                    if (last_v[s] >= 0) wait_drain(&ctl->v_full[s], (last_v[s] / VS) & 1, drain_ns);
             }
         }
     } else if (warp == kWarpFix) {
@@ -655,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpMma) {
         if (lane == 0) {
             umma_commit(&ctl->drain);
-            wait_drain(&ctl->drain, 0, limit_ns);
+            wait_drain(&ctl->drain, 0, atflash_drain_limit_ns(limit_ns));
         }
         __syncwarp();
         tc_fence_after();

@@ -156,3 +156,16 @@ def test_decode_argument_errors(L):
     assert dec(ws=None) == -3
     assert dec(wsb=100) == -3
     assert dec(vc=ctypes.c_void_p((1 << 20) + 4)) == -6
+
+
+def test_wait_limit_and_selftest_argument_errors(L):
+    import ctypes
+    L.atflash_set_wait_limit_ms.argtypes = [ctypes.c_double]
+    L.atflash_set_wait_limit_ms.restype = ctypes.c_int
+    L.atflash_selftest_wait_timeout.argtypes = [ctypes.c_double, ctypes.c_void_p]
+    L.atflash_selftest_wait_timeout.restype = ctypes.c_int
+    for bad in (0.0, -1.0, float("nan"), 60001.0):
+        assert L.atflash_set_wait_limit_ms(bad) == -1
+    for bad in (0.0, -3.0, float("nan"), 10001.0):
+        assert L.atflash_selftest_wait_timeout(bad, None) == -1  # rejected before any launch
+    assert L.atflash_set_wait_limit_ms(2000.0) == 0
