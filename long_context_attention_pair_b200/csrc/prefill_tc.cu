@@ -447,7 +447,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Boundary pairs: the dense MMA included them; remove them from the
                 // cells whose distance exceeds the pair's window (jj < n - m0 - w_r).
                 if (bd.r_lo < bd.r_full) {
-                    wc.site = 10;  // the fix-up warp has staged this tile's boundary pairs
+                    // The fix-up warp has staged this tile's boundary pairs.  This wait is
+                    // skipped on tiles without boundary pairs; it is never a phase off:
+                    // S(j) was waited for above and its MMA waited for this phase, and
+                    // the stage's next phase needs this warp to release the stage first.
+                    wc.site = 10;
                     if (!(ok = mbar_wait_warp(&ctl->k_ready[ks], (j / KS) & 1, wc))) break;
                     const float4 *bst = sBnd + ks * (kMaxStagedPairs * 64);
                     for (int r = bd.r_lo; r < bd.r_full; ++r) {
