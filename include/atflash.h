@@ -155,6 +155,34 @@ int atflash_prefill_packed(const void *qpack, const void *kpack, const void *v, 
                            int Hkv, int64_t N, int D, double rope_base, double k_window, int in_dtype,
                            int out_dtype, float *lse, cudaStream_t stream);
 
+/*
+ * Windowed prefill of a ragged batch packed along the token axis (the
+ * "variable-length" form): sequence b is tokens cu_seqlens[b] ..
+ * cu_seqlens[b+1]-1, each with its own positions 0..len_b-1 and its own causal
+ * attention; no token attends across a sequence boundary.  Same method,
+ * window and numerics as atflash_prefill ("The idea"; the window is applied
+ * per sequence with n - m measured inside the sequence).
+ *   q          [total][Hq][D] bf16, un-rotated;  k, v  [total][Hkv][D] bf16.
+ *   out        [total][Hq][D], bf16 (out_dtype ATFLASH_BF16) or fp32.
+ *   cu_seqlens device int32 [B+1]: cu[0] = 0, non-decreasing, cu[B] = total.
+ *              A sequence whose entries break these rules gets no output rows.
+ *   max_seqlen host value >= every sequence length (grid size and window
+ *              clamp); rows of longer sequences beyond it are not computed.
+ *   D in {64, 128}; Hq % Hkv == 0.
+ *   lse        NULL, or [Hq][total] fp32 (natural log-sum-exp per row).
+ *   workspace  NULL (the library takes atflash_prefill_varlen_workspace_bytes
+ *              from its stream-ordered pool for the call), or a caller buffer
+ *              of at least that size, 256-byte aligned.
+ * Errors: ATFLASH_ERR_INVALID_ARG (null pointer, shapes, total < max_seqlen),
+ * ATFLASH_ERR_UNSUPPORTED (D, out_dtype), ATFLASH_ERR_ALIGNMENT,
+ * ATFLASH_ERR_WORKSPACE; nothing is launched on error.
+ */
+int atflash_prefill_varlen(const void *q, const void *k, const void *v, void *out, const int32_t *cu_seqlens, int B,
+                           int64_t max_seqlen, int64_t total, int Hq, int Hkv, int D, double rope_base,
+                           double k_window, int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+size_t atflash_prefill_varlen_workspace_bytes(int Hq, int Hkv, int64_t total, int D);
+
 /* Device scratch bytes atflash_decode needs (0 on invalid arguments). */
 size_t atflash_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D);
 

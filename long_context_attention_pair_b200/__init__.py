@@ -71,8 +71,12 @@ def lib():
         L.atflash_rope_pack_bytes.restype = sz
         L.atflash_prefill_packed.argtypes = [vp, vp, vp, vp, i, i, i, i64, i, d, d, i, i, vp, vp]
         L.atflash_device_status.argtypes = [i]
+        L.atflash_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, i, i64, i64, i, i, i, d, d, i, vp, vp, sz, vp]
+        L.atflash_prefill_varlen_workspace_bytes.argtypes = [i, i, i64, i]
+        L.atflash_prefill_varlen_workspace_bytes.restype = sz
         for f in ("atflash_window_table", "atflash_pruned_terms", "atflash_prefill", "atflash_prefill_ex",
-                  "atflash_decode", "atflash_device_status", "atflash_rope_pack", "atflash_prefill_packed"):
+                  "atflash_decode", "atflash_device_status", "atflash_rope_pack", "atflash_prefill_packed",
+                  "atflash_prefill_varlen"):
             getattr(L, f).restype = i
         _lib = L
     return _lib
@@ -164,6 +168,37 @@ def prefill(q, k, v, rope_base: float, k_window: float = math.inf, *, out=None, 
                                   _dev(lse, "lse") if lse is not None else None, _dev(workspace, "workspace"),
                                   need, _stream_ptr(stream))
     _check(st, "atflash_prefill_ex")
+    return (out, lse) if return_lse else out
+
+
+def prefill_varlen(q, k, v, cu_seqlens, max_seqlen: int, rope_base: float, k_window: float = math.inf, *,
+                   out=None, out_dtype=None, return_lse: bool = False, workspace=None, stream=None):
+    """Windowed causal RoPE prefill of a ragged batch packed along the token axis.
+
+    q [total, Hq, D], k/v [total, Hkv, D] bf16 (un-rotated); cu_seqlens int32 [B+1]
+    on the device (sequence b is tokens cu[b]..cu[b+1]-1, positions restart at 0);
+    max_seqlen >= every sequence length.  Returns out [total, Hq, D] and, with
+    ``return_lse``, lse [Hq, total] fp32.
+    """
+    torch = _torch()
+    total, Hq, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    if out is None:
+        out = torch.empty((total, Hq, D), dtype=out_dtype if out_dtype is not None else q.dtype, device=q.device)
+    lse = torch.empty((Hq, total), dtype=torch.float32, device=q.device) if return_lse else None
+    need = int(lib().atflash_prefill_varlen_workspace_bytes(Hq, Hkv, total, D))
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    st = lib().atflash_prefill_varlen(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
+                                      _dev(cu_seqlens, "cu_seqlens"), B, int(max_seqlen), total, Hq, Hkv, D,
+                                      float(rope_base), float(k_window), _dtype_code(out),
+                                      _dev(lse, "lse") if lse is not None else None, ws_ptr,
+                                      ws_bytes if workspace is not None else need, _stream_ptr(stream))
+    _check(st, "atflash_prefill_varlen")
     return (out, lse) if return_lse else out
 
 

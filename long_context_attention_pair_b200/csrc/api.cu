@@ -266,6 +266,63 @@ int atflash_prefill(const void *q, const void *k, const void *v, void *out, int 
     return rc;
 }
 
+static int check_varlen(int B, int Hq, int Hkv, int64_t max_seqlen, int64_t total, int D, double base, double k,
+                        int out_dtype) {
+    int rc = check_shape(B, Hq, Hkv, max_seqlen);
+    if (rc != ATFLASH_OK) return rc;
+    if (total < 1 || total > INT32_MAX || max_seqlen > total) return ATFLASH_ERR_INVALID_ARG;
+    if ((rc = check_window_args(D, base, k)) != ATFLASH_OK) return rc;
+    if (D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
+    if (out_dtype != ATFLASH_F32 && out_dtype != ATFLASH_BF16) return ATFLASH_ERR_UNSUPPORTED;
+    return ATFLASH_OK;
+}
+
+size_t atflash_prefill_varlen_workspace_bytes(int Hq, int Hkv, int64_t total, int D) {
+    if (Hq < 1 || Hkv < 1 || total < 1 || total > INT32_MAX || (D != 64 && D != 128)) return 0;
+    return align256((size_t)Hq * total * D * 2) + align256((size_t)Hkv * total * D * 2);
+}
+
+int atflash_prefill_varlen(const void *q, const void *k, const void *v, void *out, const int32_t *cu_seqlens, int B,
+                           int64_t max_seqlen, int64_t total, int Hq, int Hkv, int D, double rope_base,
+                           double k_window, int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+    if (!q || !k || !v || !out || !cu_seqlens) return ATFLASH_ERR_INVALID_ARG;
+    int rc = check_varlen(B, Hq, Hkv, max_seqlen, total, D, rope_base, k_window, out_dtype);
+    if (rc != ATFLASH_OK) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATFLASH_ERR_ALIGNMENT;
+    const size_t need = atflash_prefill_varlen_workspace_bytes(Hq, Hkv, total, D);
+    void *owned = nullptr;
+    if (!workspace) {  // no caller workspace: take it from the library's stream-ordered pool
+        cudaMemPool_t pool = scratch_pool();
+        if (!pool) return ATFLASH_ERR_CUDA;
+        if (cudaMallocFromPoolAsync(&owned, need, pool, stream) != cudaSuccess) return ATFLASH_ERR_CUDA;
+        workspace = owned;
+    } else if (workspace_bytes < need) {
+        return ATFLASH_ERR_WORKSPACE;
+    } else if (reinterpret_cast<uintptr_t>(workspace) & 255u) {
+        return ATFLASH_ERR_ALIGNMENT;
+    }
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *qt = ws;
+    void *kt = ws + align256((size_t)Hq * total * D * 2);
+    WindowParams wp;
+    rc = fill_window(wp, D, rope_base, k_window, max_seqlen);
+    cudaError_t e = cudaSuccess;
+    int *status = device_status_word();
+    if (rc == ATFLASH_OK && !status) rc = ATFLASH_ERR_CUDA;
+    if (rc == ATFLASH_OK) {
+        e = launch_rope_pack_bf16(q, qt, 1, total, Hq, D, wp, stream, cu_seqlens, B);
+        if (e == cudaSuccess) e = launch_rope_pack_bf16(k, kt, 1, total, Hkv, D, wp, stream, cu_seqlens, B);
+        Problem p{B, Hq, Hkv, D, max_seqlen};
+        if (e == cudaSuccess)
+            e = launch_prefill_tc(qt, kt, v, out, out_dtype == ATFLASH_F32, lse, p, wp, status, wait_limit_ns(),
+                                  stream, cu_seqlens, total);
+        if (e != cudaSuccess) rc = ATFLASH_ERR_CUDA;
+    }
+    if (owned) cudaFreeAsync(owned, stream);
+    return rc;
+}
+
 size_t atflash_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D) {
     if (check_shape(B, Hq, Hkv, Nmax) != ATFLASH_OK || (D != 64 && D != 128)) return 0;
     return decode_workspace_bytes(B, Hq, Hkv, Nmax, D);

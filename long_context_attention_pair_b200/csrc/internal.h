@@ -32,8 +32,11 @@ struct Problem {
 // kernels read.  bf16 path: packed [b*H+h][D/16][N][16] bf16, pair-interleaved
 // (element 2j of chunk c is x~_{8c+j}, element 2j+1 is x~_{8c+j+D/2}).
 // fp32 path: [b*H+h][N][D] fp32 pair-interleaved.
+// cu (device, nseq + 1 entries) != nullptr: the token axis holds several
+// sequences and each token is rotated by its position within its sequence.
 cudaError_t launch_rope_pack_bf16(const void *x, void *y, int B, int64_t N, int Hx, int D,
-                                  const WindowParams &wp, cudaStream_t s);
+                                  const WindowParams &wp, cudaStream_t s, const int32_t *cu = nullptr,
+                                  int nseq = 0);
 cudaError_t launch_rope_pack_f32(const void *x, void *y, int B, int64_t N, int Hx, int D,
                                  const WindowParams &wp, cudaStream_t s);
 
@@ -42,9 +45,13 @@ cudaError_t launch_prefill_simt_f32(const float *qt, const float *kt, const floa
                                     float *lse, const Problem &p, const WindowParams &wp, cudaStream_t s);
 
 // tcgen05 prefill over the packed bf16 Q~/K~ and the caller's bf16 V.
+// cu_seqlens (device, B + 1 entries) != nullptr: q/k/v/out and the packed
+// Q~/K~ hold a batch of `total` tokens packed along the token axis; p.N is the
+// longest sequence.
 cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *v, void *out, int out_f32,
                               float *lse, const Problem &p, const WindowParams &wp, int *status,
-                              uint64_t wait_limit_ns, cudaStream_t s);
+                              uint64_t wait_limit_ns, cudaStream_t s, const int32_t *cu_seqlens = nullptr,
+                              int64_t total = 0);
 
 // Split-KV decode + merge.
 int decode_split_keys(int B, int Hkv, int64_t Nmax);

@@ -159,12 +159,15 @@ __device__ __forceinline__ bool wait_drain(uint64_t *bar, uint32_t parity, uint6
     return true;
 }
 
-template <int D>
+// kVarlen: the batch is packed along the token axis (q, k, v, out [total][H][D],
+// packed Q~/K~ [H][D/16][total][16]); sequence b holds tokens cu[b]..cu[b+1]-1
+// and N is the longest sequence.  Otherwise q/k/v/out are [B][N][H][D].
+template <int D, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ WindowParams wp,
                       void *out, int out_f32, float *lse, int64_t N, int Hq, int Hkv, int *status,
-                      uint64_t limit_ns) {
+                      uint64_t limit_ns, const int32_t *cu_seqlens, int64_t total) {
     using F = Cfg<D>;
     constexpr int C = F::C;
     constexpr int H = D / 2;
@@ -191,6 +194,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nwg = two ? 2 : 1;
     const int64_t n0 = (int64_t)qt * kBM;
     const int nkt = qt + 1;  // key tiles 0..qt (causal)
+    // Where this CTA's sequence lives: first token on the token axis, valid rows,
+    // batch coordinate of the tensor maps, rows per batch of out / lse.
+    int64_t tokbase = 0, seq_len = N, nrows = N;
+    int bz = b;
+    if constexpr (kVarlen) {
+        const int64_t t0 = cu_seqlens[b], t1 = cu_seqlens[b + 1];
+        // A malformed table selects no rows (every write below stays inside [0, total)).
+        seq_len = (t0 >= 0 && t1 >= t0 && t1 <= total) ? t1 - t0 : 0;
+        tokbase = seq_len > 0 ? t0 : 0;
+        nrows = total;
+        bz = 0;
+        if (n0 >= seq_len) return;  // this sequence has fewer query tiles (whole CTA, before any barrier)
+    }
 
     if (threadIdx.x == 0) {
         mbar_init(&ctl->q_full, 1);
@@ -243,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_expect_tx(&ctl->q_full, (uint32_t)(nwg * F::QBytes));
             for (int t = 0; t < nwg; ++t)
                 for (int c = 0; c < C; ++c)
-                    tma_load_3d(sQ + t * F::QBytes + c * kChunkBytes, &tm_q, &ctl->q_full, 0, (int)n0,
-                                (b * Hq + h0 + t) * C + c);
+                    tma_load_3d(sQ + t * F::QBytes + c * kChunkBytes, &tm_q, &ctl->q_full, 0, (int)(tokbase + n0),
+                                (bz * Hq + h0 + t) * C + c);
             bool ok = true;
             BandWalk bw;
             bw.init(w, H, n0);
@@ -256,15 +272,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!(ok = mbar_wait(&ctl->k_empty[ks], ((j / KS) & 1) ^ 1, wc))) break;
                 mbar_expect_tx(&ctl->k_full[ks], (uint32_t)(C - ca) * kChunkBytes);
                 for (int c = ca; c < C; ++c)
-                    tma_load_3d(sK + ks * F::KBytes + c * kChunkBytes, &tm_k, &ctl->k_full[ks], 0, (int)m0,
-                                (b * Hkv + kvh) * C + c);
+                    tma_load_3d(sK + ks * F::KBytes + c * kChunkBytes, &tm_k, &ctl->k_full[ks], 0,
+                                (int)(tokbase + m0), (bz * Hkv + kvh) * C + c);
                 last_k[ks] = j;
                 wc.site = 2;
                 if (!(ok = mbar_wait(&ctl->v_empty[vs], ((j / VS) & 1) ^ 1, wc))) break;
                 mbar_expect_tx(&ctl->v_full[vs], F::VBytes);
                 for (int gidx = 0; gidx < D / 64; ++gidx)
                     tma_load_4d(sV + vs * F::VBytes + gidx * 16384, &tm_v, &ctl->v_full[vs], gidx * 64, kvh,
-                                (int)m0, b);
+                                (int)(tokbase + m0), bz);
                 last_v[vs] = j;
             }
             if (!ok) {
@@ -616,13 +632,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) {
                 tc_fence_after();
                 const float inv = 1.f / lrun;
-                const size_t o = ((size_t)((int64_t)b * N + n) * Hq + hq) * D;
+                const size_t o = ((size_t)((int64_t)bz * nrows + tokbase + n) * Hq + hq) * D;
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(tO + cc * 32, r);
                     tmem_ld_wait(r);
-                    if (n < N) {
+                    if (n < seq_len) {
                         if (out_f32) {
                             float4 *dst =
                                 reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + o + cc * 32);
@@ -648,8 +664,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                if (lse && n < N)
-                    lse[((size_t)b * Hq + hq) * N + n] = (m_used + __log2f(lrun)) * 0.69314718055994531f;
+                if (lse && n < seq_len)
+                    lse[((size_t)bz * Hq + hq) * nrows + tokbase + n] = (m_used + __log2f(lrun)) * 0.69314718055994531f;
             }
         }
     }
@@ -683,26 +699,30 @@ static cudaError_t make_map(CUtensorMap *map, void *base, int rank, const cuuint
 
 cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *v, void *out, int out_f32,
                               float *lse, const Problem &p, const WindowParams &wp, int *status,
-                              uint64_t wait_limit_ns, cudaStream_t s) {
+                              uint64_t wait_limit_ns, cudaStream_t s, const int32_t *cu_seqlens, int64_t total) {
     const int C = p.D / 16;
+    const bool varlen = cu_seqlens != nullptr;
+    // Token axis of the maps: N per batch entry, or the whole packed batch.
+    const cuuint64_t T = varlen ? (cuuint64_t)total : (cuuint64_t)p.N;
+    const cuuint64_t NB = varlen ? 1 : (cuuint64_t)p.B;
     CUtensorMap tq, tk, tv;
     {
-        cuuint64_t dims[3] = {16, (cuuint64_t)p.N, (cuuint64_t)p.B * p.Hq * C};
-        cuuint64_t str[2] = {32, (cuuint64_t)p.N * 32};
+        cuuint64_t dims[3] = {16, T, NB * p.Hq * C};
+        cuuint64_t str[2] = {32, T * 32};
         cuuint32_t box[3] = {16, tc::kBM, 1};
         cudaError_t e = make_map(&tq, const_cast<void *>(qpack), 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B);
         if (e != cudaSuccess) return e;
     }
     {
-        cuuint64_t dims[3] = {16, (cuuint64_t)p.N, (cuuint64_t)p.B * p.Hkv * C};
-        cuuint64_t str[2] = {32, (cuuint64_t)p.N * 32};
+        cuuint64_t dims[3] = {16, T, NB * p.Hkv * C};
+        cuuint64_t str[2] = {32, T * 32};
         cuuint32_t box[3] = {16, tc::kBN, 1};
         cudaError_t e = make_map(&tk, const_cast<void *>(kpack), 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B);
         if (e != cudaSuccess) return e;
     }
     {
-        cuuint64_t dims[4] = {(cuuint64_t)p.D, (cuuint64_t)p.Hkv, (cuuint64_t)p.N, (cuuint64_t)p.B};
-        cuuint64_t str[3] = {(cuuint64_t)p.D * 2, (cuuint64_t)p.Hkv * p.D * 2, (cuuint64_t)p.N * p.Hkv * p.D * 2};
+        cuuint64_t dims[4] = {(cuuint64_t)p.D, (cuuint64_t)p.Hkv, T, NB};
+        cuuint64_t str[3] = {(cuuint64_t)p.D * 2, (cuuint64_t)p.Hkv * p.D * 2, T * p.Hkv * p.D * 2};
         cuuint32_t box[4] = {64, 1, tc::kBN, 1};
         cudaError_t e = make_map(&tv, const_cast<void *>(v), 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (e != cudaSuccess) return e;
@@ -711,21 +731,24 @@ cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *
     const int G = p.Hq / p.Hkv;
     dim3 grid((unsigned)num_qt, (unsigned)(p.B * p.Hkv * ((G + 1) / 2)));
     cudaError_t e;
+#define ATF_PREFILL_TC(DD, VL)                                                                                   \
+    do {                                                                                                         \
+        const int smem = tc::Cfg<DD>::Request;                                                                  \
+        e = cudaFuncSetAttribute(tc::prefill_tc_kernel<DD, VL>, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
+                                 smem);                                                                          \
+        if (e != cudaSuccess) return e;                                                                          \
+        tc::prefill_tc_kernel<DD, VL><<<grid, tc::kThreads, smem, s>>>(tq, tk, tv, wp, out, out_f32, lse, p.N,  \
+                                                                       p.Hq, p.Hkv, status, wait_limit_ns,     \
+                                                                       cu_seqlens, total);                     \
+    } while (0)
     if (p.D == 128) {
-        const int smem = tc::Cfg<128>::Request;
-        e = cudaFuncSetAttribute(tc::prefill_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        tc::prefill_tc_kernel<128><<<grid, tc::kThreads, smem, s>>>(tq, tk, tv, wp, out, out_f32, lse, p.N, p.Hq,
-                                                                    p.Hkv, status, wait_limit_ns);
+        if (varlen) ATF_PREFILL_TC(128, true); else ATF_PREFILL_TC(128, false);
     } else if (p.D == 64) {
-        const int smem = tc::Cfg<64>::Request;
-        e = cudaFuncSetAttribute(tc::prefill_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        tc::prefill_tc_kernel<64><<<grid, tc::kThreads, smem, s>>>(tq, tk, tv, wp, out, out_f32, lse, p.N, p.Hq,
-                                                                   p.Hkv, status, wait_limit_ns);
+        if (varlen) ATF_PREFILL_TC(64, true); else ATF_PREFILL_TC(64, false);
     } else {
         return cudaErrorInvalidValue;
     }
+#undef ATF_PREFILL_TC
     return cudaGetLastError();
 }
 

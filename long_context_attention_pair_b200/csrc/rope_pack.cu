@@ -29,18 +29,34 @@ __device__ __forceinline__ float2 rope_cos_sin(int64_t n, double theta) {
     return make_float2(c, s);
 }
 
+// Position of token n of a batch packed along the token axis: n minus the start
+// of its sequence (cu[s] <= n < cu[s+1]); the token's own index without cu.
+__device__ __forceinline__ int64_t token_position(int64_t n, const int32_t *cu, int nseq) {
+    if (!cu) return n;
+    int lo = 0, hi = nseq;  // largest s with cu[s] <= n
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if ((int64_t)cu[mid] <= n) lo = mid; else hi = mid;
+    }
+    return n - (int64_t)cu[lo];
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) rope_pack_bf16_kernel(const __nv_bfloat16 *__restrict__ x,
                                                              __nv_bfloat16 *__restrict__ y, int64_t N, int Hx,
-                                                             const __grid_constant__ WindowParams wp) {
+                                                             const __grid_constant__ WindowParams wp,
+                                                             const int32_t *__restrict__ cu, int nseq) {
     constexpr int H = D / 2;
     constexpr int C = D / 16;
     __shared__ float2 cs[H][kRopePos];
+    __shared__ int64_t pos[kRopePos];
     const int b = blockIdx.y;
     const int64_t n0 = (int64_t)blockIdx.x * kRopePos;
+    if (threadIdx.x < kRopePos) pos[threadIdx.x] = token_position(n0 + threadIdx.x, cu, nseq);
+    __syncthreads();
     for (int e = threadIdx.x; e < H * kRopePos; e += blockDim.x) {
         int r = e / kRopePos, p = e % kRopePos;
-        cs[r][p] = (n0 + p < N) ? rope_cos_sin(n0 + p, wp.theta[r]) : make_float2(1.f, 0.f);
+        cs[r][p] = (n0 + p < N) ? rope_cos_sin(pos[p], wp.theta[r]) : make_float2(1.f, 0.f);
     }
     __syncthreads();
     const int p = threadIdx.x & 31;
@@ -96,12 +112,14 @@ __global__ void __launch_bounds__(256) rope_pack_f32_kernel(const float *__restr
 }
 
 cudaError_t launch_rope_pack_bf16(const void *x, void *y, int B, int64_t N, int Hx, int D,
-                                  const WindowParams &wp, cudaStream_t s) {
+                                  const WindowParams &wp, cudaStream_t s, const int32_t *cu, int nseq) {
     dim3 grid((unsigned)((N + kRopePos - 1) / kRopePos), (unsigned)B);
     if (D == 128)
-        rope_pack_bf16_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)x, (__nv_bfloat16 *)y, N, Hx, wp);
+        rope_pack_bf16_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)x, (__nv_bfloat16 *)y, N, Hx, wp,
+                                                        cu, nseq);
     else if (D == 64)
-        rope_pack_bf16_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)x, (__nv_bfloat16 *)y, N, Hx, wp);
+        rope_pack_bf16_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)x, (__nv_bfloat16 *)y, N, Hx, wp, cu,
+                                                       nseq);
     else
         return cudaErrorInvalidValue;
     return cudaGetLastError();

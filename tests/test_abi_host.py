@@ -169,3 +169,26 @@ def test_wait_limit_and_selftest_argument_errors(L):
     for bad in (0.0, -3.0, float("nan"), 10001.0):
         assert L.atflash_selftest_wait_timeout(bad, None) == -1  # rejected before any launch
     assert L.atflash_set_wait_limit_ms(2000.0) == 0
+
+
+def test_varlen_argument_errors(L):
+    import ctypes
+    vp = ctypes.c_void_p(4096)
+
+    def call(**kw):
+        a = dict(q=vp, k=vp, v=vp, out=vp, cu=vp, B=2, maxs=100, total=150, Hq=4, Hkv=2, D=128, base=1e4,
+                 kwin=8.0, outd=atf.BF16, lse=None, ws=vp, wsb=1 << 40)
+        a.update(kw)
+        return L.atflash_prefill_varlen(a["q"], a["k"], a["v"], a["out"], a["cu"], a["B"], a["maxs"], a["total"],
+                                        a["Hq"], a["Hkv"], a["D"], a["base"], a["kwin"], a["outd"], a["lse"],
+                                        a["ws"], a["wsb"], None)
+    assert call(cu=None) == -1
+    assert call(total=50) == -1          # shorter than max_seqlen
+    assert call(B=0) == -1
+    assert call(Hq=3) == -1
+    assert call(D=80) == -2
+    assert call(outd=7) == -2
+    assert call(q=ctypes.c_void_p(4098)) == -6
+    assert call(wsb=10) == -3
+    assert atf.lib().atflash_prefill_varlen_workspace_bytes(4, 2, 150, 128) > 0
+    assert atf.lib().atflash_prefill_varlen_workspace_bytes(4, 2, 150, 96) == 0
