@@ -183,6 +183,30 @@ int atflash_prefill_varlen(const void *q, const void *k, const void *v, void *ou
                            cudaStream_t stream);
 size_t atflash_prefill_varlen_workspace_bytes(int Hq, int Hkv, int64_t total, int D);
 
+/*
+ * Decode over a paged KV cache (the layout serving engines keep): pages of
+ * page_size tokens in one pool; keys i*page_size .. (i+1)*page_size-1 of
+ * sequence b are in page block_table[b*max_pages + i].  Same method, window,
+ * numerics, q/out layouts and splits as atflash_decode (bf16 caches only).
+ *   page_size   a multiple of 64 (one 64-key TMA stage never straddles a page).
+ *   kv_layout   ATFLASH_KV_NHD: kpages and vpages [num_pages][page_size][Hkv][D]
+ *               bf16 (K rotated iff kcache_rotated);
+ *               ATFLASH_KV_PACKED: kpages [num_pages][Hkv][D/16][page_size][16]
+ *               bf16, rotated, in the packed chunk layout (kcache_rotated = 1),
+ *               vpages as for NHD.
+ *   block_table device int32 [B][max_pages]; seqlens device int32 [B],
+ *               1 <= seqlens[b] <= max_pages*page_size.  A page index past
+ *               the row or an id outside [0, num_pages) reads zeros.
+ *   workspace   >= atflash_decode_workspace_bytes(B, Hq, Hkv,
+ *               max_pages*page_size, D) bytes, 16-byte aligned.
+ * Errors as atflash_decode, plus ATFLASH_ERR_INVALID_ARG for page_size,
+ * max_pages, num_pages or kv_layout.
+ */
+int atflash_decode_paged(const void *q, const void *kpages, const void *vpages, const int32_t *block_table,
+                         const int32_t *seqlens, void *out, int B, int Hq, int Hkv, int max_pages, int num_pages,
+                         int page_size, int D, double rope_base, double k_window, int kcache_rotated, int kv_layout,
+                         int out_dtype, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Device scratch bytes atflash_decode needs (0 on invalid arguments). */
 size_t atflash_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D);
 

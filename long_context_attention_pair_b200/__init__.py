@@ -74,9 +74,10 @@ def lib():
         L.atflash_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, i, i64, i64, i, i, i, d, d, i, vp, vp, sz, vp]
         L.atflash_prefill_varlen_workspace_bytes.argtypes = [i, i, i64, i]
         L.atflash_prefill_varlen_workspace_bytes.restype = sz
+        L.atflash_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, d, d, i, i, i, vp, sz, vp]
         for f in ("atflash_window_table", "atflash_pruned_terms", "atflash_prefill", "atflash_prefill_ex",
                   "atflash_decode", "atflash_device_status", "atflash_rope_pack", "atflash_prefill_packed",
-                  "atflash_prefill_varlen"):
+                  "atflash_prefill_varlen", "atflash_decode_paged"):
             getattr(L, f).restype = i
         _lib = L
     return _lib
@@ -200,6 +201,36 @@ def prefill_varlen(q, k, v, cu_seqlens, max_seqlen: int, rope_base: float, k_win
                                       ws_bytes if workspace is not None else need, _stream_ptr(stream))
     _check(st, "atflash_prefill_varlen")
     return (out, lse) if return_lse else out
+
+
+def decode_paged(q, kpages, vpages, block_table, seqlens, page_size: int, rope_base: float,
+                 k_window: float = math.inf, *, kcache_rotated: bool = False, kv_layout: str = "NHD", out=None,
+                 out_dtype=None, workspace=None, stream=None):
+    """One decode step over a paged KV cache.
+
+    q [B, Hq, D] bf16; block_table int32 [B, max_pages]; seqlens int32 [B].
+    kv_layout "NHD": kpages/vpages [num_pages, page_size, Hkv, D];
+    "PACKED": kpages [num_pages, Hkv, D/16, page_size, 16] (rotated), vpages as NHD.
+    page_size must be a multiple of 64.  Returns out [B, Hq, D].
+    """
+    torch = _torch()
+    B, Hq, D = q.shape
+    num_pages = vpages.shape[0]
+    Hkv = vpages.shape[2]
+    max_pages = block_table.shape[1]
+    lay = {"NHD": KV_NHD, "PACKED": KV_PACKED}[kv_layout]
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=out_dtype if out_dtype is not None else q.dtype, device=q.device)
+    need = decode_workspace_bytes(B, Hq, Hkv, max_pages * page_size, D)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib().atflash_decode_paged(_dev(q, "q"), _dev(kpages, "kpages"), _dev(vpages, "vpages"),
+                                    _dev(block_table, "block_table"), _dev(seqlens, "seqlens"), _dev(out, "out"), B,
+                                    Hq, Hkv, max_pages, num_pages, int(page_size), D, float(rope_base),
+                                    float(k_window), 1 if kcache_rotated else 0, lay, _dtype_code(out),
+                                    _dev(workspace, "workspace"), need, _stream_ptr(stream))
+    _check(st, "atflash_decode_paged")
+    return out
 
 
 def rope_pack(x, rope_base: float, *, out=None, stream=None):

@@ -328,6 +328,36 @@ size_t atflash_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int 
     return decode_workspace_bytes(B, Hq, Hkv, Nmax, D);
 }
 
+int atflash_decode_paged(const void *q, const void *kpages, const void *vpages, const int32_t *block_table,
+                         const int32_t *seqlens, void *out, int B, int Hq, int Hkv, int max_pages, int num_pages,
+                         int page_size, int D, double rope_base, double k_window, int kcache_rotated, int kv_layout,
+                         int out_dtype, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (!q || !kpages || !vpages || !block_table || !seqlens || !out) return ATFLASH_ERR_INVALID_ARG;
+    if (max_pages < 1 || num_pages < 1 || page_size < 64 || page_size % 64 != 0) return ATFLASH_ERR_INVALID_ARG;
+    const int64_t Nmax = (int64_t)max_pages * page_size;
+    int rc = check_shape(B, Hq, Hkv, Nmax);
+    if (rc != ATFLASH_OK) return rc;
+    if ((int64_t)num_pages * Hkv * (D / 16) > INT32_MAX) return ATFLASH_ERR_INVALID_ARG;
+    if ((rc = check_window_args(D, rope_base, k_window)) != ATFLASH_OK) return rc;
+    if (kcache_rotated != 0 && kcache_rotated != 1) return ATFLASH_ERR_INVALID_ARG;
+    if (kv_layout != ATFLASH_KV_NHD && kv_layout != ATFLASH_KV_PACKED) return ATFLASH_ERR_INVALID_ARG;
+    if (kv_layout == ATFLASH_KV_PACKED && !kcache_rotated) return ATFLASH_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
+    if (out_dtype != ATFLASH_F32 && out_dtype != ATFLASH_BF16) return ATFLASH_ERR_UNSUPPORTED;
+    if (Hq / Hkv > 16) return ATFLASH_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(kpages) || !aligned16(vpages) || !aligned16(out)) return ATFLASH_ERR_ALIGNMENT;
+    const size_t need = decode_workspace_bytes(B, Hq, Hkv, Nmax, D);
+    if (!workspace || workspace_bytes < need) return ATFLASH_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return ATFLASH_ERR_ALIGNMENT;
+    WindowParams wp;
+    if ((rc = fill_window(wp, D, rope_base, k_window, Nmax)) != ATFLASH_OK) return rc;
+    Problem p{B, Hq, Hkv, D, Nmax};
+    PagedKV pk{block_table, max_pages, page_size, num_pages};
+    cudaError_t e = launch_decode(q, kpages, vpages, seqlens, out, out_dtype == ATFLASH_F32, 0, kcache_rotated,
+                                  kv_layout, p, wp, static_cast<float *>(workspace), stream, &pk);
+    return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
+}
+
 int atflash_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out,
                    int B, int Hq, int Hkv, int64_t Nmax, int D, double rope_base, double k_window,
                    int kcache_rotated, int kv_layout, int in_dtype, int out_dtype, void *workspace,

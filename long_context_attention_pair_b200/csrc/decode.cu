@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float
 
 cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const int32_t *seqlens, void *out,
                           int out_f32, int in_f32, int krot, int layout, const Problem &p, const WindowParams &wp,
-                          float *workspace, cudaStream_t s) {
+                          float *workspace, cudaStream_t s, const PagedKV *paged) {
     const int nhd = (layout == ATFLASH_KV_NHD);
     const int split_keys = decode_split_keys(p.B, p.Hkv, p.N);
     const int nsplit = decode_num_splits(p.B, p.Hkv, p.N);
@@ -254,9 +254,9 @@ cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const i
         int *status = device_status_word();
         if (!status) return cudaErrorUnknown;
         e = launch_decode_tc(q, kc, vc, seqlens, krot, layout, p, wp, workspace, split_keys, nsplit, status,
-                             wait_limit_ns(), s);
+                             wait_limit_ns(), s, paged);
     } else {
-        if (layout == ATFLASH_KV_PACKED) return cudaErrorInvalidValue;  // packed caches are bf16
+        if (layout == ATFLASH_KV_PACKED || paged) return cudaErrorInvalidValue;  // bf16 caches only
         dim3 grid((unsigned)nsplit, (unsigned)p.Hkv, (unsigned)p.B);
         dim3 block(32 * kDecodeWarps);
         if (p.D == 128)

@@ -116,11 +116,15 @@ __device__ __forceinline__ void mask_pairs(uint32_t &lo, uint32_t &hi, bool keep
 // The natural-layout kernel (rotation at load) is asked for two CTAs per SM, which
 // lets the compiler use more registers than its default; the packed kernel keeps
 // the default, which measured faster.
-template <int D, bool kPacked>
+// kPaged: K and V live in pages of page_size tokens (a multiple of the 64-key
+// stage), page block_table[b * max_pages + i] holding keys i*page_size.. of
+// sequence b; the maps index pages along their outermost axis.
+template <int D, bool kPacked, bool kPaged>
 __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const void *q_,
     const int32_t *__restrict__ seqlens, float *__restrict__ ws, int Hq, int Hkv, int nhd, int krot, int split_keys,
-    int nsplit, const __grid_constant__ WindowParams wp, int *status, uint64_t limit_ns) {
+    int nsplit, const __grid_constant__ WindowParams wp, int *status, uint64_t limit_ns,
+    const int32_t *__restrict__ block_table, int max_pages, int page_size, int num_pages) {
     using F = Cfg<D>;
     constexpr int H = F::H, C = F::C;
     constexpr int kStages = F::kStages;
@@ -197,7 +201,26 @@ __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
                 const uint32_t bytes = (uint32_t)(C - c_lo) * 2048u + (uint32_t)F::VBytes;
                 mbar_expect_tx(&bars->full[st], bytes);
                 uint8_t *kst = sK + st * F::KBytes;
-                if (kPacked) {
+                if constexpr (kPaged) {
+                    // A stage never straddles a page (page_size is a multiple of 64).  A
+                    // page index past the table row or an id outside the pool becomes -1,
+                    // which the maps treat as out of bounds (zero fill, no access).
+                    const int64_t pi = k0 / page_size;
+                    int page = pi < max_pages ? block_table[(size_t)b * max_pages + pi] : -1;
+                    if (page < 0 || page >= num_pages) page = -1;
+                    const int kk = (int)(k0 % page_size);
+                    if (kPacked) {
+                        for (int c = c_lo; c < C; ++c)
+                            tma_load_3d(kst + c * 2048, &tm_k, &bars->full[st], 0, kk, (page * Hkv + g) * C + c);
+                    } else {
+                        for (int c = c_lo; c < C; ++c)
+                            for (int hf = 0; hf < 2; ++hf)
+                                tma_load_4d(kst + (2 * c + hf) * 1024, &tm_k, &bars->full[st], hf * H + 8 * c, g, kk,
+                                            page);
+                    }
+                    for (int gi = 0; gi < D / 64; ++gi)
+                        tma_load_4d(sV + st * F::VBytes + gi * 8192, &tm_v, &bars->full[st], 64 * gi, g, kk, page);
+                } else if (kPacked) {
                     for (int c = c_lo; c < C; ++c)
                         tma_load_3d(kst + c * 2048, &tm_k, &bars->full[st], 0, (int)k0, (b * Hkv + g) * C + c);
                 } else {
@@ -209,10 +232,12 @@ __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
                             else tma_load_3d(dst, &tm_k, &bars->full[st], x, (int)k0, b * Hkv + g);
                         }
                 }
-                for (int gi = 0; gi < D / 64; ++gi) {
-                    uint8_t *dst = sV + st * F::VBytes + gi * 8192;
-                    if (nhd) tma_load_4d(dst, &tm_v, &bars->full[st], 64 * gi, g, (int)k0, b);
-                    else tma_load_3d(dst, &tm_v, &bars->full[st], 64 * gi, (int)k0, b * Hkv + g);
+                if constexpr (!kPaged) {
+                    for (int gi = 0; gi < D / 64; ++gi) {
+                        uint8_t *dst = sV + st * F::VBytes + gi * 8192;
+                        if (nhd) tma_load_4d(dst, &tm_v, &bars->full[st], 64 * gi, g, (int)k0, b);
+                        else tma_load_3d(dst, &tm_v, &bars->full[st], 64 * gi, (int)k0, b * Hkv + g);
+                    }
                 }
             }
             __syncwarp();
@@ -515,13 +540,30 @@ static cudaError_t make_map_bf16(CUtensorMap *map, const void *base, int rank, c
 
 cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, const int32_t *seqlens, int krot,
                              int layout, const Problem &p, const WindowParams &wp, float *workspace, int split_keys,
-                             int nsplit, int *status, uint64_t limit_ns, cudaStream_t s) {
+                             int nsplit, int *status, uint64_t limit_ns, cudaStream_t s, const PagedKV *paged) {
     CUtensorMap tk, tv;
     const cuuint64_t Dd = (cuuint64_t)p.D, Nm = (cuuint64_t)p.N, Hk = (cuuint64_t)p.Hkv, Bb = (cuuint64_t)p.B;
     const int nhd = (layout == ATFLASH_KV_NHD);
     const bool packed = (layout == ATFLASH_KV_PACKED);
     cudaError_t e;
-    if (packed) {
+    if (paged) {
+        // Pools: V [num_pages][page_size][Hkv][D]; K the same (natural, rotated or
+        // not) or packed [num_pages][Hkv][D/16][page_size][16].
+        const cuuint64_t P = (cuuint64_t)paged->page_size, NP = (cuuint64_t)paged->num_pages;
+        cuuint64_t dv[4] = {Dd, Hk, P, NP};
+        cuuint64_t sv[3] = {Dd * 2, Hk * Dd * 2, P * Hk * Dd * 2};
+        cuuint32_t boxv[4] = {64, 1, dtc::kStageKeys, 1};
+        if ((e = make_map_bf16(&tv, vc, 4, dv, sv, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
+        if (packed) {
+            cuuint64_t dk[3] = {16, P, NP * Hk * (Dd / 16)};
+            cuuint64_t sk[2] = {32, P * 32};
+            cuuint32_t boxk[3] = {16, dtc::kStageKeys, 1};
+            if ((e = make_map_bf16(&tk, kc, 3, dk, sk, boxk, CU_TENSOR_MAP_SWIZZLE_32B)) != cudaSuccess) return e;
+        } else {
+            cuuint32_t boxk[4] = {8, 1, dtc::kStageKeys, 1};
+            if ((e = make_map_bf16(&tk, kc, 4, dv, sv, boxk, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess) return e;
+        }
+    } else if (packed) {
         // K: [B*Hkv*D/16][Nmax][16] packed chunks; V: [B][Hkv][Nmax][D].
         cuuint64_t dk[3] = {16, Nm, Bb * Hk * (Dd / 16)};
         cuuint64_t sk[2] = {32, Nm * 32};
@@ -545,20 +587,31 @@ cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, cons
         if ((e = make_map_bf16(&tv, vc, 3, dims, str, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
     }
     dim3 grid((unsigned)nsplit, (unsigned)p.Hkv, (unsigned)p.B);
-#define ATF_DEC_TC(DD, PK)                                                                                     \
+    const int32_t *bt = paged ? paged->block_table : nullptr;
+    const int maxp = paged ? paged->max_pages : 0, psz = paged ? paged->page_size : 0;
+    const int npool = paged ? paged->num_pages : 0;
+#define ATF_DEC_TC(DD, PK, PG)                                                                                 \
     do {                                                                                                       \
         const int smem = dtc::Cfg<DD>::Request;                                                                \
-        if ((e = cudaFuncSetAttribute(dtc::decode_tc_kernel<DD, PK>,                                          \
+        if ((e = cudaFuncSetAttribute(dtc::decode_tc_kernel<DD, PK, PG>,                                      \
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)      \
             return e;                                                                                          \
-        dtc::decode_tc_kernel<DD, PK><<<grid, dtc::kThreads, smem, s>>>(tk, tv, q, seqlens, workspace, p.Hq,   \
-                                                                        p.Hkv, nhd, krot, split_keys, nsplit, \
-                                                                        wp, status, limit_ns);                 \
+        dtc::decode_tc_kernel<DD, PK, PG><<<grid, dtc::kThreads, smem, s>>>(                                  \
+            tk, tv, q, seqlens, workspace, p.Hq, p.Hkv, nhd, krot, split_keys, nsplit, wp, status, limit_ns,  \
+            bt, maxp, psz, npool);                                                                             \
     } while (0)
     if (p.D == 128) {
-        if (packed) ATF_DEC_TC(128, true); else ATF_DEC_TC(128, false);
+        if (paged) {
+            if (packed) ATF_DEC_TC(128, true, true); else ATF_DEC_TC(128, false, true);
+        } else {
+            if (packed) ATF_DEC_TC(128, true, false); else ATF_DEC_TC(128, false, false);
+        }
     } else {
-        if (packed) ATF_DEC_TC(64, true); else ATF_DEC_TC(64, false);
+        if (paged) {
+            if (packed) ATF_DEC_TC(64, true, true); else ATF_DEC_TC(64, false, true);
+        } else {
+            if (packed) ATF_DEC_TC(64, true, false); else ATF_DEC_TC(64, false, false);
+        }
     }
 #undef ATF_DEC_TC
     return cudaGetLastError();

@@ -57,9 +57,16 @@ cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *
 int decode_split_keys(int B, int Hkv, int64_t Nmax);
 int decode_num_splits(int B, int Hkv, int64_t Nmax);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D);
+// A paged KV cache: keys i*page_size.. of sequence b are in pool page
+// block_table[b*max_pages + i]; page_size is a multiple of 64.
+struct PagedKV {
+    const int32_t *block_table;  // device, [B][max_pages]
+    int max_pages, page_size, num_pages;
+};
 cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, const int32_t *seqlens, int krot,
                              int layout, const Problem &p, const WindowParams &wp, float *workspace, int split_keys,
-                             int nsplit, int *status, uint64_t limit_ns, cudaStream_t s);
+                             int nsplit, int *status, uint64_t limit_ns, cudaStream_t s,
+                             const PagedKV *paged = nullptr);
 
 // Device status word of the current device (bounded waits record timeouts
 // here) and the wait limit in nanoseconds.
@@ -69,7 +76,8 @@ uint64_t wait_limit_ns();
 cudaError_t launch_selftest_wait(int *status, uint64_t limit_ns, cudaStream_t s);
 cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const int32_t *seqlens, void *out,
                           int out_f32, int in_f32, int krot, int layout, const Problem &p,
-                          const WindowParams &wp, float *workspace, cudaStream_t s);
+                          const WindowParams &wp, float *workspace, cudaStream_t s,
+                          const PagedKV *paged = nullptr);
 
 // Driver entry point for cuTensorMapEncodeTiled (resolved once, no libcuda link).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,

@@ -192,3 +192,27 @@ def test_varlen_argument_errors(L):
     assert call(wsb=10) == -3
     assert atf.lib().atflash_prefill_varlen_workspace_bytes(4, 2, 150, 128) > 0
     assert atf.lib().atflash_prefill_varlen_workspace_bytes(4, 2, 150, 96) == 0
+
+
+def test_paged_decode_argument_errors(L):
+    import ctypes
+    vp = ctypes.c_void_p(4096)
+
+    def call(**kw):
+        a = dict(q=vp, kp=vp, vpg=vp, bt=vp, sl=vp, out=vp, B=2, Hq=8, Hkv=2, mp=16, npool=40, page=64, D=128,
+                 base=1e7, kwin=16.0, krot=0, lay=atf.KV_NHD, outd=atf.F32, ws=vp, wsb=1 << 40)
+        a.update(kw)
+        return L.atflash_decode_paged(a["q"], a["kp"], a["vpg"], a["bt"], a["sl"], a["out"], a["B"], a["Hq"],
+                                      a["Hkv"], a["mp"], a["npool"], a["page"], a["D"], a["base"], a["kwin"],
+                                      a["krot"], a["lay"], a["outd"], a["ws"], a["wsb"], None)
+    assert call(bt=None) == -1
+    assert call(page=48) == -1            # not a multiple of 64
+    assert call(page=0) == -1
+    assert call(mp=0) == -1
+    assert call(npool=0) == -1
+    assert call(lay=atf.KV_HND) == -1     # pages are NHD or packed
+    assert call(lay=atf.KV_PACKED, krot=0) == -1
+    assert call(D=96) == -2
+    assert call(Hq=34, Hkv=2) == -2       # more than 16 query heads per KV head
+    assert call(ws=None) == -3
+    assert call(kp=ctypes.c_void_p(4100)) == -6
