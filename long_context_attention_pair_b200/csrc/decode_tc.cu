@@ -14,15 +14,23 @@
 // The contraction order inside a K-step is [8 low-half dims, 8 high-half dims]
 // for both Q~ and K~, so every dot product is unchanged.
 //
-// Angles: the producer writes, per stage, the base angle stage_start*theta_r
-// reduced mod 2*pi in fp64; a key at offset i adds i*theta_r (i < 64) in fp32,
-// reduces once more and takes sin/cos on [-pi, pi].
+// Angles (rotation at load only): the producer writes, per stage, the base
+// angle stage_start*theta_r reduced mod 2*pi, from a 64-bit fixed-point turn
+// count: theta_r/(2*pi) as a fraction of 2^64, times the integer position,
+// wraps modulo 2^64 = whole turns, so the reduction is exact integer
+// arithmetic (the fraction carries fp64's precision of theta_r).  A key at
+// offset i adds i*theta_r (i < 64) in fp32, reduces once more and takes
+// sin/cos on [-pi, pi].
 //
 // Packed cache (ATFLASH_KV_PACKED): K already rotated and stored as the RoPE
 // pre-pass writes it, [B*Hkv][D/16][Nmax][16] with 8 frequency pairs per 32-byte
 // chunk.  A pruned chunk of 64 keys is then 2 KB of HBM that is never fetched;
 // in the natural layouts a key's pruned dims are a short prefix of each 128-byte
-// half and HBM's access granularity fetches them anyway.
+// half and HBM's access granularity fetches them anyway.  The 2 KB of one chunk
+// of a stage are contiguous, so the copy views them as 16 rows of 128 bytes
+// (4 keys per row, SWIZZLE_128B) rather than 64 rows of 32 bytes: a quarter of
+// the TMA row requests, which bound the producer otherwise.  That view needs
+// Nmax % 4 == 0 (whole rows per chunk); other lengths keep the 32-byte rows.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -44,7 +52,9 @@ struct Cfg {
     static constexpr int kStages = 3;
     static constexpr int H = D / 2;
     static constexpr int C = D / 16;                   // chunks of 8 pairs
-    static constexpr int KBytes = C * 2 * 1024;        // [c][half][64 keys][8 dims] bf16
+    // K stage: packed [c][64 keys][32 B] (SW128 as 16 rows of 128 B, or SW32), natural
+    // [D/64][64 keys][64 dims] SW128 like V.
+    static constexpr int KBytes = C * 2 * 1024;
     static constexpr int VBytes = (D / 64) * 8192;     // [D/64][64 keys][64 dims] bf16, SW128
     static constexpr int OffK = 0;
     static constexpr int OffV = OffK + kStages * KBytes;
@@ -60,15 +70,6 @@ struct Bars {
     uint64_t full[kMaxStages], empty[kMaxStages];
     int abort_flag;
 };
-
-__device__ __forceinline__ int first_kept_pair(const int *w, int H, int64_t d) {
-    int lo = 0, hi = H;
-    while (lo < hi) {
-        int mid = (lo + hi) >> 1;
-        if ((int64_t)w[mid] >= d) hi = mid; else lo = mid + 1;
-    }
-    return lo;
-}
 
 // r*(d) as d shrinks: keys of later stages are nearer the query, so the first
 // kept pair only moves down; amortised O(1) per stage.
@@ -86,6 +87,13 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &d0, uint32_t 
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(d0), "=r"(d1), "=r"(d2), "=r"(d3)
                  : "r"(addr));
+}
+// 8x8 transpose of a b16 matrix held one row pair per thread (thread t: row t/4,
+// columns 2(t%4), 2(t%4)+1); afterwards thread t holds row t/4 of the transpose.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
 }
 __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -119,12 +127,13 @@ __device__ __forceinline__ void mask_pairs(uint32_t &lo, uint32_t &hi, bool keep
 // kPaged: K and V live in pages of page_size tokens (a multiple of the 64-key
 // stage), page block_table[b * max_pages + i] holding keys i*page_size.. of
 // sequence b; the maps index pages along their outermost axis.
-template <int D, bool kPacked, bool kPaged>
+// NT: tiles of 8 query heads (a GQA group of G <= 8 heads takes one tile, up to 16 two).
+template <int D, bool kPacked, bool kPaged, int NT>
 __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const void *q_,
     const int32_t *__restrict__ seqlens, float *__restrict__ ws, int Hq, int Hkv, int nhd, int krot, int split_keys,
     int nsplit, const __grid_constant__ WindowParams wp, int *status, uint64_t limit_ns,
-    const int32_t *__restrict__ block_table, int max_pages, int page_size, int num_pages) {
+    const int32_t *__restrict__ block_table, int max_pages, int page_size, int num_pages, int k_rows128) {
     using F = Cfg<D>;
     constexpr int H = F::H, C = F::C;
     constexpr int kStages = F::kStages;
@@ -137,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
     Bars *bars = reinterpret_cast<Bars *>(smem + F::OffBar);
     __shared__ int sw[kMaxPairs];
     __shared__ float sTheta[kMaxPairs];
+    __shared__ uint64_t sTurn[kMaxPairs];  // theta_r / (2*pi) in units of 2^-64 turns
 
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_);
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -158,6 +168,8 @@ __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
     for (int r = threadIdx.x; r < H; r += kThreads) {
         sw[r] = wp.w[r];
         sTheta[r] = (float)wp.theta[r];
+        // theta_r <= 1, so the fraction is below 2^61.4 and fits the integer.
+        sTurn[r] = __double2ull_rn(wp.theta[r] * (0.15915494309189533576888376337251 * 18446744073709551616.0));
     }
     // Rotated queries at position L-1 (fp64 angle reduction), rows >= G are zero.
     for (int e = threadIdx.x; e < 16 * H; e += kThreads) {
@@ -184,21 +196,35 @@ __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
         bool ok = true;
         int last[kMaxStages];
         for (int s = 0; s < kMaxStages; ++s) last[s] = -1;
+        if (lane == 0) {
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+        }
+        // Only a rotation at load needs the stage base angles.
+        const bool rotate = !kPacked && !krot;
+        // r*(d) of the stage's nearest key: stages move towards the query, so the
+        // first kept pair only moves down (amortised O(1) per stage).
+        int r_near = H;
         for (int it = 0; it < nstage && ok; ++it) {
             const int st = it % kStages;
             const int64_t k0 = s0 + (int64_t)it * kStageKeys;
             int64_t k1 = k0 + kStageKeys - 1;
             if (k1 > s1 - 1) k1 = s1 - 1;
-            const int c_lo = first_kept_pair(sw, H, (L - 1) - k1) >> 3;  // nearest key keeps the most
+            r_near = walk_down(sw, r_near, (int)((L - 1) - k1));  // nearest key keeps the most
+            const int c_lo = r_near >> 3;
             if (!(ok = mbar_wait_warp(&bars->empty[st], ((it / kStages) & 1) ^ 1, wc))) break;
-            for (int r = lane; r < H; r += 32) {
-                double turns = (double)k0 * wp.theta[r] * 0.15915494309189533576888376337251;
-                turns -= rint(turns);
-                sBase[st * H + r] = (float)(turns * 6.283185307179586476925286766559);
+            if (rotate) {
+                for (int r = lane; r < H; r += 32) {
+                    // Turns of k0 * theta_r modulo 1, as a signed fraction of 2^64 in [-1/2, 1/2).
+                    const int64_t t = (int64_t)((uint64_t)k0 * sTurn[r]);
+                    sBase[st * H + r] = (float)t * 3.4061215800865545e-19f;  // 2*pi / 2^64
+                }
             }
             __syncwarp();
             if (lane == 0) {
-                const uint32_t bytes = (uint32_t)(C - c_lo) * 2048u + (uint32_t)F::VBytes;
+                // Natural layouts fetch whole K rows (their pruned dims cost DRAM sectors anyway).
+                const uint32_t kbytes = kPacked ? (uint32_t)(C - c_lo) * 2048u : (uint32_t)F::KBytes;
+                const uint32_t bytes = kbytes + (uint32_t)F::VBytes;
                 mbar_expect_tx(&bars->full[st], bytes);
                 uint8_t *kst = sK + st * F::KBytes;
                 if constexpr (kPaged) {
@@ -210,27 +236,26 @@ __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
                     if (page < 0 || page >= num_pages) page = -1;
                     const int kk = (int)(k0 % page_size);
                     if (kPacked) {
+                        // Pages hold a multiple of 64 keys, so the 128-byte row view always applies.
                         for (int c = c_lo; c < C; ++c)
-                            tma_load_3d(kst + c * 2048, &tm_k, &bars->full[st], 0, kk, (page * Hkv + g) * C + c);
+                            tma_load_3d(kst + c * 2048, &tm_k, &bars->full[st], 0, kk / 4, (page * Hkv + g) * C + c);
                     } else {
-                        for (int c = c_lo; c < C; ++c)
-                            for (int hf = 0; hf < 2; ++hf)
-                                tma_load_4d(kst + (2 * c + hf) * 1024, &tm_k, &bars->full[st], hf * H + 8 * c, g, kk,
-                                            page);
+                        for (int gi = 0; gi < D / 64; ++gi)
+                            tma_load_4d(kst + gi * 8192, &tm_k, &bars->full[st], 64 * gi, g, kk, page);
                     }
                     for (int gi = 0; gi < D / 64; ++gi)
                         tma_load_4d(sV + st * F::VBytes + gi * 8192, &tm_v, &bars->full[st], 64 * gi, g, kk, page);
                 } else if (kPacked) {
+                    const int ky = k_rows128 ? (int)(k0 / 4) : (int)k0;
                     for (int c = c_lo; c < C; ++c)
-                        tma_load_3d(kst + c * 2048, &tm_k, &bars->full[st], 0, (int)k0, (b * Hkv + g) * C + c);
+                        tma_load_3d(kst + c * 2048, &tm_k, &bars->full[st], 0, ky, (b * Hkv + g) * C + c);
                 } else {
-                    for (int c = c_lo; c < C; ++c)
-                        for (int hf = 0; hf < 2; ++hf) {
-                            uint8_t *dst = kst + (2 * c + hf) * 1024;
-                            const int x = hf * H + 8 * c;
-                            if (nhd) tma_load_4d(dst, &tm_k, &bars->full[st], x, g, (int)k0, b);
-                            else tma_load_3d(dst, &tm_k, &bars->full[st], x, (int)k0, b * Hkv + g);
-                        }
+                    // 64 keys x 64 dims per box, SWIZZLE_128B, like V.
+                    for (int gi = 0; gi < D / 64; ++gi) {
+                        uint8_t *dst = kst + gi * 8192;
+                        if (nhd) tma_load_4d(dst, &tm_k, &bars->full[st], 64 * gi, g, (int)k0, b);
+                        else tma_load_3d(dst, &tm_k, &bars->full[st], 64 * gi, (int)k0, b * Hkv + g);
+                    }
                 }
                 if constexpr (!kPaged) {
                     for (int gi = 0; gi < D / 64; ++gi) {
@@ -253,31 +278,45 @@ __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
         }
     } else {
         // ----------------------------------------------------------- consumers
-        const int gq = lane >> 2, tq = lane & 3;  // mma fragment row group / column pair
-        // Q~ A-fragments per chunk: k-order [dims 8c..8c+7, dims H+8c..H+8c+7].
-        uint32_t qa[C][4];
+        // Keys are the M rows of mma.sync m16n8k16 and the query heads of the group
+        // its N columns (NT tiles of 8 heads): S^T = K~ Q~^T and O^T += V^T P^T.  A
+        // group has at most 16 heads, so no head rows are padded beyond the tile.
+        // Thread (gq, tq) = (lane / 4, lane % 4) holds S^T of keys gq and gq + 8 and
+        // of heads 8t + 2tq, 8t + 2tq + 1 of head tile t.
+        const int gq = lane >> 2, tq = lane & 3;
+        // Q~^T B-fragments per chunk and head tile (head 8t + gq): elements
+        // k = 2tq, 2tq+1 and k = 8+2tq, 9+2tq of the chunk's contraction order.
+        uint32_t qb[C][NT][2];
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            if (kPacked) {
-                // k-order of a packed chunk: (pair 8c+e/2, component e%2).
-                const int pa = 8 * c + tq, pb = pa + 4;
-                qa[c][0] = pack_bf16x2(sQ[gq * D + pa], sQ[gq * D + pa + H]);
-                qa[c][1] = pack_bf16x2(sQ[(gq + 8) * D + pa], sQ[(gq + 8) * D + pa + H]);
-                qa[c][2] = pack_bf16x2(sQ[gq * D + pb], sQ[gq * D + pb + H]);
-                qa[c][3] = pack_bf16x2(sQ[(gq + 8) * D + pb], sQ[(gq + 8) * D + pb + H]);
-            } else {
-                const int lo = 8 * c + 2 * tq, hi = H + 8 * c + 2 * tq;
-                qa[c][0] = pack_bf16x2(sQ[gq * D + lo], sQ[gq * D + lo + 1]);
-                qa[c][1] = pack_bf16x2(sQ[(gq + 8) * D + lo], sQ[(gq + 8) * D + lo + 1]);
-                qa[c][2] = pack_bf16x2(sQ[gq * D + hi], sQ[gq * D + hi + 1]);
-                qa[c][3] = pack_bf16x2(sQ[(gq + 8) * D + hi], sQ[(gq + 8) * D + hi + 1]);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const float *qrow = sQ + (8 * t + gq) * D;
+                if (kPacked) {
+                    // k-order of a packed chunk: (pair 8c + k/2, component k%2).
+                    const int pa = 8 * c + tq, pb = pa + 4;
+                    qb[c][t][0] = pack_bf16x2(qrow[pa], qrow[pa + H]);
+                    qb[c][t][1] = pack_bf16x2(qrow[pb], qrow[pb + H]);
+                } else {
+                    // k-order [dims 8c..8c+7, dims H+8c..H+8c+7].
+                    const int lo = 8 * c + 2 * tq, hi = H + 8 * c + 2 * tq;
+                    qb[c][t][0] = pack_bf16x2(qrow[lo], qrow[lo + 1]);
+                    qb[c][t][1] = pack_bf16x2(qrow[hi], qrow[hi + 1]);
+                }
             }
         }
         const float scale_log2 = 1.4426950408889634f * rsqrtf((float)D);
-        float o[D / 8][4];
+        // O^T accumulators: dims 16dg + gq (e = 0, 1) and 16dg + gq + 8 (e = 2, 3),
+        // heads 8t + 2tq (e even) and 8t + 2tq + 1 (e odd).
+        float o[D / 16][NT][4];
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};  // rows gq, gq+8
+        for (int i = 0; i < D / 16; ++i)
+#pragma unroll
+            for (int t = 0; t < NT; ++t) o[i][t][0] = o[i][t][1] = o[i][t][2] = o[i][t][3] = 0.f;
+        // Running max (log2 units) and this thread's part of the sum, per head 8t + 2tq + hh.
+        float m_run[NT][2], l_run[NT][2];
+#pragma unroll
+        for (int t = 0; t < NT; ++t) m_run[t][0] = m_run[t][1] = -INFINITY, l_run[t][0] = l_run[t][1] = 0.f;
         const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
         bool ok = true;
         // Positions fit in int32 (Nmax <= 2^31 - 1).  Walk pointers for r*(d) of the
@@ -295,159 +334,169 @@ __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
             const int k1 = (k0 + kStageKeys - 1 < kend) ? k0 + kStageKeys - 1 : kend;
             r_stage = walk_down(sw, r_stage, Lq - k1);
             const int c_stage = r_stage >> 3;
-            float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            float sodd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            float sacc[NT][4], sodd[NT][4];
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sacc[t][e] = sodd[t][e] = 0.f;
             if (kw0 < (int)s1) {
                 r_warp = walk_down(sw, r_warp, Lq - kw1);
                 r_keep = walk_down(sw, r_keep, Lq - kw0);
                 const int c_warp = r_warp >> 3;
-                // Keys of this thread's fragments: n-tile 0 -> kw0 + gq, n-tile 1 -> kw0 + 8 + gq.
+                // Distances of this thread's keys kw0 + gq and kw0 + gq + 8.
                 const int da = Lq - (kw0 + gq), db = da - 8;
                 const float fa = (float)(16 * wq + gq), fb = fa + 8.f;
                 const uint32_t kst = sKa + st * F::KBytes;
                 const int mi = lane >> 3, ri = lane & 7;
                 const int c_keep = (r_keep + 7) >> 3;
+                // ldmatrix x4 of a chunk gives, per thread, b0 = key gq / first 8 k,
+                // b1 = key gq / last 8 k, b2 = key gq+8 / first 8 k, b3 = key gq+8 /
+                // last 8 k; the A fragment of the 16 keys is (b0, b2, b1, b3).
                 if constexpr (kPacked) {
                     const int c_begin = c_warp > c_stage ? c_warp : c_stage;
                     // All of this warp's K fragments first (independent shared-memory loads in
                     // flight together), then the masks and the MMAs.
                     uint32_t kb[C][4];
+                    // Matrix mi of the x4 load: keys +8*(mi>>1), bytes 16*(mi&1) of each key's 32.
+                    const int key = 16 * wq + 8 * (mi >> 1) + ri;
+                    // 128-byte rows (4 keys each, SWIZZLE_128B: 16-byte unit ^= row & 7), or
+                    // 32-byte rows (one key each, SWIZZLE_32B: unit bit 0 ^= key bit 2).
+                    const uint32_t koff =
+                        (kPaged || k_rows128)
+                            ? (uint32_t)((key >> 2) * 128 + ((((key & 3) * 2 + (mi & 1)) ^ ((key >> 2) & 7)) << 4))
+                            : (uint32_t)(key * 32 + ((16 * (mi & 1)) ^ ((key & 4) << 2)));
 #pragma unroll
                     for (int c = 0; c < C; ++c) {
                         if (c < c_begin) continue;
-                        // 64 keys x 32 B per chunk, SWIZZLE_32B; matrix mi: keys +8*(mi>>1), bytes 16*(mi&1).
-                        const int key = 16 * wq + 8 * (mi >> 1) + ri;
-                        ldsm_x4(kst + c * 2048 + key * 32 + ((16 * (mi & 1)) ^ ((key & 4) << 2)), kb[c][0], kb[c][1],
-                                kb[c][2], kb[c][3]);
+                        ldsm_x4(kst + c * 2048 + koff, kb[c][0], kb[c][1], kb[c][2], kb[c][3]);
                     }
 #pragma unroll
                     for (int c = 0; c < C; ++c) {
                         if (c < c_begin) continue;
                         // Chunks from c_keep on are kept by every key of this warp: no masking.
                         const bool masked = c < c_keep;
-                        uint32_t b0 = kb[c][0], b1 = kb[c][1], b2 = kb[c][2], b3 = kb[c][3];
+                        uint32_t a[4] = {kb[c][0], kb[c][2], kb[c][1], kb[c][3]};
                         if (masked) {
                             const int p0 = 8 * c + tq, p1 = p0 + 4;
                             const int w0 = sw[p0], w1 = sw[p1];
-                            b0 = (da <= w0) ? b0 : 0u;
-                            b1 = (da <= w1) ? b1 : 0u;
-                            b2 = (db <= w0) ? b2 : 0u;
-                            b3 = (db <= w1) ? b3 : 0u;
+                            a[0] = (da <= w0) ? a[0] : 0u;
+                            a[2] = (da <= w1) ? a[2] : 0u;
+                            a[1] = (db <= w0) ? a[1] : 0u;
+                            a[3] = (db <= w1) ? a[3] : 0u;
                         }
                         // Two independent accumulation chains (chunk parity).
-                        if (c & 1) {
-                            mma16816(sodd[0], qa[c], b0, b1);
-                            mma16816(sodd[1], qa[c], b2, b3);
-                        } else {
-                            mma16816(sacc[0], qa[c], b0, b1);
-                            mma16816(sacc[1], qa[c], b2, b3);
+#pragma unroll
+                        for (int t = 0; t < NT; ++t) {
+                            if (c & 1) mma16816(sodd[t], a, qb[c][t][0], qb[c][t][1]);
+                            else mma16816(sacc[t], a, qb[c][t][0], qb[c][t][1]);
                         }
                     }
                 } else {
-                    for (int c = (c_warp > c_stage ? c_warp : c_stage); c < C; ++c) {
+#pragma unroll
+                    for (int c = 0; c < C; ++c) {
+                        if (c < (c_warp > c_stage ? c_warp : c_stage)) continue;
                         const bool masked = c < c_keep;
                         uint32_t b0, b1, b2, b3;
-                        if (kPacked) {
-                            // 64 keys x 32 B per chunk, SWIZZLE_32B; matrix mi: keys +8*(mi>>1), bytes 16*(mi&1).
-                            const int key = 16 * wq + 8 * (mi >> 1) + ri;
-                            ldsm_x4(kst + c * 2048 + key * 32 + ((16 * (mi & 1)) ^ ((key & 4) << 2)), b0, b1, b2, b3);
+                        // Rows of 64 dims (128 B, SWIZZLE_128B: 16-byte unit ^= key & 7); matrix
+                        // mi: keys +8*(mi>>1), dims (mi&1)*H + 8c .. +8 of each key.
+                        const int key = 16 * wq + 8 * (mi >> 1) + ri;
+                        const int dim0 = (mi & 1) * H + 8 * c;
+                        const uint32_t addr =
+                            kst + (dim0 >> 6) * 8192 + key * 128 + ((((dim0 & 63) >> 3) ^ (key & 7)) << 4);
+                        ldsm_x4(addr, b0, b1, b2, b3);
+                        const int p0 = 8 * c + 2 * tq, p1 = p0 + 1;
+                        const int w0 = sw[p0], w1 = sw[p1];
+                        const bool ka0 = da <= w0, ka1 = da <= w1, kb0 = db <= w0, kb1 = db <= w1;
+                        if (krot) {
                             if (masked) {
-                                const int p0 = 8 * c + tq, p1 = p0 + 4;
-                                const int w0 = sw[p0], w1 = sw[p1];
-                                b0 = (da <= w0) ? b0 : 0u;
-                                b1 = (da <= w1) ? b1 : 0u;
-                                b2 = (db <= w0) ? b2 : 0u;
-                                b3 = (db <= w1) ? b3 : 0u;
+                                mask_pairs(b0, b1, ka0, ka1);
+                                mask_pairs(b2, b3, kb0, kb1);
                             }
                         } else {
-                            const uint32_t addr = kst + (2 * c + (mi & 1)) * 1024 + (16 * wq + 8 * (mi >> 1) + ri) * 16;
-                            ldsm_x4(addr, b0, b1, b2, b3);
-                            const int p0 = 8 * c + 2 * tq, p1 = p0 + 1;
-                            const int w0 = sw[p0], w1 = sw[p1];
-                            const bool ka0 = da <= w0, ka1 = da <= w1, kb0 = db <= w0, kb1 = db <= w1;
-                            if (krot) {
-                                if (masked) {
-                                    mask_pairs(b0, b1, ka0, ka1);
-                                    mask_pairs(b2, b3, kb0, kb1);
-                                }
-                            } else {
-                                const float th0 = sTheta[p0], th1 = sTheta[p1];
-                                const float base0 = sBase[st * H + p0], base1 = sBase[st * H + p1];
-                                float ang[4] = {fmaf(fa, th0, base0), fmaf(fa, th1, base1), fmaf(fb, th0, base0),
-                                                fmaf(fb, th1, base1)};
-                                float cs[4], sn[4];
+                            const float th0 = sTheta[p0], th1 = sTheta[p1];
+                            const float base0 = sBase[st * H + p0], base1 = sBase[st * H + p1];
+                            float ang[4] = {fmaf(fa, th0, base0), fmaf(fa, th1, base1), fmaf(fb, th0, base0),
+                                            fmaf(fb, th1, base1)};
+                            float cs[4], sn[4];
 #pragma unroll
-                                for (int u = 0; u < 4; ++u) {
-                                    const float turns = rintf(ang[u] * 0.15915494309189533577f);
-                                    const float x = fmaf(-turns, 6.283185307179586477f, ang[u]);
-                                    __sincosf(x, &sn[u], &cs[u]);
-                                }
-                                rotate_pairs(b0, b1, cs[0], sn[0], cs[1], sn[1], ka0, ka1);
-                                rotate_pairs(b2, b3, cs[2], sn[2], cs[3], sn[3], kb0, kb1);
+                            for (int u = 0; u < 4; ++u) {
+                                const float turns = rintf(ang[u] * 0.15915494309189533577f);
+                                const float x = fmaf(-turns, 6.283185307179586477f, ang[u]);
+                                __sincosf(x, &sn[u], &cs[u]);
                             }
+                            rotate_pairs(b0, b1, cs[0], sn[0], cs[1], sn[1], ka0, ka1);
+                            rotate_pairs(b2, b3, cs[2], sn[2], cs[3], sn[3], kb0, kb1);
                         }
-                        // Two independent accumulation chains (chunk parity).
-                        if (c & 1) {
-                            mma16816(sodd[0], qa[c], b0, b1);
-                            mma16816(sodd[1], qa[c], b2, b3);
-                        } else {
-                            mma16816(sacc[0], qa[c], b0, b1);
-                            mma16816(sacc[1], qa[c], b2, b3);
+                        const uint32_t a[4] = {b0, b2, b1, b3};
+#pragma unroll
+                        for (int t = 0; t < NT; ++t) {
+                            if (c & 1) mma16816(sodd[t], a, qb[c][t][0], qb[c][t][1]);
+                            else mma16816(sacc[t], a, qb[c][t][0], qb[c][t][1]);
                         }
                     }
                 }
 #pragma unroll
+                for (int t = 0; t < NT; ++t)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sacc[t][e] += sodd[t][e];
+            }
+            // Online softmax over this warp's 16 keys, per head: the thread's two keys,
+            // then the 8 row groups (lanes with the same tq).
+            float x[NT][4];
+            float alpha[NT][2];
+            bool rescale = false;
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                float tmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    sacc[0][e] += sodd[0][e];
-                    sacc[1][e] += sodd[1][e];
+                    const int key = kw0 + gq + 8 * (e >> 1);
+                    const float v = (key < (int)s1) ? sacc[t][e] * scale_log2 : -INFINITY;
+                    x[t][e] = v;
+                    tmax[e & 1] = fmaxf(tmax[e & 1], v);
+                }
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    tmax[hh] = fmaxf(tmax[hh], __shfl_xor_sync(0xffffffffu, tmax[hh], 4));
+                    tmax[hh] = fmaxf(tmax[hh], __shfl_xor_sync(0xffffffffu, tmax[hh], 8));
+                    tmax[hh] = fmaxf(tmax[hh], __shfl_xor_sync(0xffffffffu, tmax[hh], 16));
+                    const bool need = tmax[hh] > m_run[t][hh] + kRescaleThreshold;
+                    const float m_new = need ? tmax[hh] : m_run[t][hh];
+                    alpha[t][hh] = need ? fast_exp2(m_run[t][hh] - m_new) : 1.f;
+                    rescale |= need;
+                    m_run[t][hh] = m_new;
                 }
             }
-            // Online softmax over this warp's 16 keys; rows gq (sacc[.][0..1]) and gq+8 ([2..3]).
-            float x[2][4];
-            float tmax[2] = {-INFINITY, -INFINITY};
+            uint32_t pb[NT][2];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int key = kw0 + 8 * nt + 2 * tq + (e & 1);
-                    const float v = (key < (int)s1) ? sacc[nt][e] * scale_log2 : -INFINITY;
-                    x[nt][e] = v;
-                    tmax[e >> 1] = fmaxf(tmax[e >> 1], v);
-                }
-            float alpha[2];
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                tmax[rr] = fmaxf(tmax[rr], __shfl_xor_sync(0xffffffffu, tmax[rr], 1));
-                tmax[rr] = fmaxf(tmax[rr], __shfl_xor_sync(0xffffffffu, tmax[rr], 2));
-                const bool need = tmax[rr] > m_run[rr] + kRescaleThreshold;
-                const float m_new = need ? tmax[rr] : m_run[rr];
-                alpha[rr] = need ? fast_exp2(m_run[rr] - m_new) : 1.f;
-                m_run[rr] = m_new;
+            for (int t = 0; t < NT; ++t) {
+                const float mref0 = m_run[t][0] == -INFINITY ? 0.f : m_run[t][0];
+                const float mref1 = m_run[t][1] == -INFINITY ? 0.f : m_run[t][1];
+                const float p0 = fast_exp2(x[t][0] - mref0), p1 = fast_exp2(x[t][1] - mref1);
+                const float p2 = fast_exp2(x[t][2] - mref0), p3 = fast_exp2(x[t][3] - mref1);
+                l_run[t][0] = l_run[t][0] * alpha[t][0] + (p0 + p2);
+                l_run[t][1] = l_run[t][1] * alpha[t][1] + (p1 + p3);
+                // P^T (keys x heads) into the B fragment of O^T += V^T P^T: an 8x8
+                // transpose per key half turns (key gq; heads 2tq, 2tq+1) into
+                // (head gq; keys 2tq, 2tq+1).
+                pb[t][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+                pb[t][1] = movmatrix_trans(pack_bf16x2(p2, p3));
             }
-            float p[2][4];
-            const float mref[2] = {m_run[0] == -INFINITY ? 0.f : m_run[0], m_run[1] == -INFINITY ? 0.f : m_run[1]};
+            if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+                for (int i = 0; i < D / 16; ++i)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) p[nt][e] = fast_exp2(x[nt][e] - mref[e >> 1]);
-            l_run[0] = l_run[0] * alpha[0] + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
-            l_run[1] = l_run[1] * alpha[1] + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
-            if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
-#pragma unroll
-                for (int i = 0; i < D / 8; ++i) {
-                    o[i][0] *= alpha[0];
-                    o[i][1] *= alpha[0];
-                    o[i][2] *= alpha[1];
-                    o[i][3] *= alpha[1];
-                }
+                    for (int t = 0; t < NT; ++t) {
+                        o[i][t][0] *= alpha[t][0];
+                        o[i][t][1] *= alpha[t][1];
+                        o[i][t][2] *= alpha[t][0];
+                        o[i][t][3] *= alpha[t][1];
+                    }
             }
-            uint32_t pa[4];
-            pa[0] = pack_bf16x2(p[0][0], p[0][1]);
-            pa[1] = pack_bf16x2(p[0][2], p[0][3]);
-            pa[2] = pack_bf16x2(p[1][0], p[1][1]);
-            pa[3] = pack_bf16x2(p[1][2], p[1][3]);
             if (kw0 < (int)s1) {
-                // O += P V: V rows = this warp's 16 keys, SW128 rows of 64 dims.
+                // O^T += V^T P^T: V rows = this warp's 16 keys, SW128 rows of 64 dims.
+                // ldmatrix.trans matrix mi: keys 8*(mi&1).., dims 16dg + 8*(mi>>1)..; the
+                // A fragment (dims x keys) of 16 dims is (v0, v2, v1, v3).
                 const uint32_t vst = sVa + st * F::VBytes;
                 const int mi = lane >> 3, ri = lane & 7;
                 const int vkey = 16 * wq + 8 * (mi & 1) + ri;
@@ -459,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
                     ldsm_x4_t(addr, v0, v1, v2, v3);
                     if (kw0 + 15 >= (int)s1) {
                         // Rows past the sequence end may hold anything: P is 0 there, and
-                        // 0 * (non-finite) must not reach O.  b0b1: keys 2tq, 2tq+1; b2b3: +8.
+                        // 0 * (non-finite) must not reach O.  v0, v2: keys 2tq, 2tq+1; v1, v3: +8.
                         const int kk = kw0 + 2 * tq, se = (int)s1;
                         const uint32_t m01 = (kk < se ? 0x0000FFFFu : 0u) | (kk + 1 < se ? 0xFFFF0000u : 0u);
                         const uint32_t m89 = (kk + 8 < se ? 0x0000FFFFu : 0u) | (kk + 9 < se ? 0xFFFF0000u : 0u);
@@ -468,35 +517,45 @@ __global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
                         v2 &= m01;
                         v3 &= m89;
                     }
-                    mma16816(o[2 * dg], pa, v0, v1);
-                    mma16816(o[2 * dg + 1], pa, v2, v3);
+                    const uint32_t a[4] = {v0, v2, v1, v3};
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) mma16816(o[dg][t], a, pb[t][0], pb[t][1]);
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->empty[st]);
         }
-        // Full row sums across the quad, then fold the four warps through shared memory.
+        // Row sums across the 8 row groups, then fold the four warps through shared memory.
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-            l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
-            l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
-        }
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                l_run[t][hh] += __shfl_xor_sync(0xffffffffu, l_run[t][hh], 4);
+                l_run[t][hh] += __shfl_xor_sync(0xffffffffu, l_run[t][hh], 8);
+                l_run[t][hh] += __shfl_xor_sync(0xffffffffu, l_run[t][hh], 16);
+            }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumers));  // consumers only: stages are drained
-        float *red = reinterpret_cast<float *>(smem);  // reuse the K/V stages: [warp][16][D+2]
+        float *red = reinterpret_cast<float *>(smem);  // reuse the K/V stages: [warp][16 heads][D+2]
         float *mine = red + (size_t)warp * 16 * (D + 2);
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
-            const int col = 8 * i + 2 * tq;
-            mine[gq * (D + 2) + 2 + col] = o[i][0];
-            mine[gq * (D + 2) + 3 + col] = o[i][1];
-            mine[(gq + 8) * (D + 2) + 2 + col] = o[i][2];
-            mine[(gq + 8) * (D + 2) + 3 + col] = o[i][3];
-        }
-        if (tq == 0) {
-            mine[gq * (D + 2)] = m_run[0];
-            mine[gq * (D + 2) + 1] = l_run[0];
-            mine[(gq + 8) * (D + 2)] = m_run[1];
-            mine[(gq + 8) * (D + 2) + 1] = l_run[1];
+        for (int i = 0; i < D / 16; ++i)
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const int h0 = 8 * t + 2 * tq, d = 16 * i + gq;
+                mine[h0 * (D + 2) + 2 + d] = o[i][t][0];
+                mine[(h0 + 1) * (D + 2) + 2 + d] = o[i][t][1];
+                mine[h0 * (D + 2) + 2 + d + 8] = o[i][t][2];
+                mine[(h0 + 1) * (D + 2) + 2 + d + 8] = o[i][t][3];
+            }
+        if (gq == 0) {
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const int h0 = 8 * t + 2 * tq;
+                mine[h0 * (D + 2)] = m_run[t][0];
+                mine[h0 * (D + 2) + 1] = l_run[t][0];
+                mine[(h0 + 1) * (D + 2)] = m_run[t][1];
+                mine[(h0 + 1) * (D + 2) + 1] = l_run[t][1];
+            }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumers));
         for (int e = threadIdx.x; e < G * D; e += 32 * kConsumers) {
@@ -545,6 +604,9 @@ cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, cons
     const cuuint64_t Dd = (cuuint64_t)p.D, Nm = (cuuint64_t)p.N, Hk = (cuuint64_t)p.Hkv, Bb = (cuuint64_t)p.B;
     const int nhd = (layout == ATFLASH_KV_NHD);
     const bool packed = (layout == ATFLASH_KV_PACKED);
+    // Packed K chunks as 128-byte rows: always for pages (a multiple of 64 keys),
+    // for a contiguous cache when every chunk holds whole rows.
+    const int rows128 = packed && (paged || (p.N % 4) == 0) ? 1 : 0;
     cudaError_t e;
     if (paged) {
         // Pools: V [num_pages][page_size][Hkv][D]; K the same (natural, rotated or
@@ -555,20 +617,27 @@ cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, cons
         cuuint32_t boxv[4] = {64, 1, dtc::kStageKeys, 1};
         if ((e = make_map_bf16(&tv, vc, 4, dv, sv, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
         if (packed) {
-            cuuint64_t dk[3] = {16, P, NP * Hk * (Dd / 16)};
-            cuuint64_t sk[2] = {32, P * 32};
-            cuuint32_t boxk[3] = {16, dtc::kStageKeys, 1};
-            if ((e = make_map_bf16(&tk, kc, 3, dk, sk, boxk, CU_TENSOR_MAP_SWIZZLE_32B)) != cudaSuccess) return e;
+            // One chunk of a page: P keys x 32 B contiguous, viewed as P/4 rows of 128 B.
+            cuuint64_t dk[3] = {64, P / 4, NP * Hk * (Dd / 16)};
+            cuuint64_t sk[2] = {128, P * 32};
+            cuuint32_t boxk[3] = {64, dtc::kStageKeys / 4, 1};
+            if ((e = make_map_bf16(&tk, kc, 3, dk, sk, boxk, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
         } else {
-            cuuint32_t boxk[4] = {8, 1, dtc::kStageKeys, 1};
-            if ((e = make_map_bf16(&tk, kc, 4, dv, sv, boxk, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess) return e;
+            if ((e = make_map_bf16(&tk, kc, 4, dv, sv, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
         }
     } else if (packed) {
         // K: [B*Hkv*D/16][Nmax][16] packed chunks; V: [B][Hkv][Nmax][D].
-        cuuint64_t dk[3] = {16, Nm, Bb * Hk * (Dd / 16)};
-        cuuint64_t sk[2] = {32, Nm * 32};
-        cuuint32_t boxk[3] = {16, dtc::kStageKeys, 1};
-        if ((e = make_map_bf16(&tk, kc, 3, dk, sk, boxk, CU_TENSOR_MAP_SWIZZLE_32B)) != cudaSuccess) return e;
+        if (rows128) {
+            cuuint64_t dk[3] = {64, Nm / 4, Bb * Hk * (Dd / 16)};
+            cuuint64_t sk[2] = {128, Nm * 32};
+            cuuint32_t boxk[3] = {64, dtc::kStageKeys / 4, 1};
+            if ((e = make_map_bf16(&tk, kc, 3, dk, sk, boxk, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
+        } else {
+            cuuint64_t dk[3] = {16, Nm, Bb * Hk * (Dd / 16)};
+            cuuint64_t sk[2] = {32, Nm * 32};
+            cuuint32_t boxk[3] = {16, dtc::kStageKeys, 1};
+            if ((e = make_map_bf16(&tk, kc, 3, dk, sk, boxk, CU_TENSOR_MAP_SWIZZLE_32B)) != cudaSuccess) return e;
+        }
         cuuint64_t dims[3] = {Dd, Nm, Bb * Hk};
         cuuint64_t str[2] = {Dd * 2, Nm * Dd * 2};
         cuuint32_t boxv[3] = {64, dtc::kStageKeys, 1};
@@ -576,29 +645,34 @@ cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, cons
     } else if (nhd) {
         cuuint64_t dims[4] = {Dd, Hk, Nm, Bb};
         cuuint64_t str[3] = {Dd * 2, Hk * Dd * 2, Nm * Hk * Dd * 2};
-        cuuint32_t boxk[4] = {8, 1, dtc::kStageKeys, 1}, boxv[4] = {64, 1, dtc::kStageKeys, 1};
-        if ((e = make_map_bf16(&tk, kc, 4, dims, str, boxk, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess) return e;
+        cuuint32_t boxv[4] = {64, 1, dtc::kStageKeys, 1};
+        if ((e = make_map_bf16(&tk, kc, 4, dims, str, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
         if ((e = make_map_bf16(&tv, vc, 4, dims, str, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
     } else {
         cuuint64_t dims[3] = {Dd, Nm, Bb * Hk};
         cuuint64_t str[2] = {Dd * 2, Nm * Dd * 2};
-        cuuint32_t boxk[3] = {8, dtc::kStageKeys, 1}, boxv[3] = {64, dtc::kStageKeys, 1};
-        if ((e = make_map_bf16(&tk, kc, 3, dims, str, boxk, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess) return e;
+        cuuint32_t boxv[3] = {64, dtc::kStageKeys, 1};
+        if ((e = make_map_bf16(&tk, kc, 3, dims, str, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
         if ((e = make_map_bf16(&tv, vc, 3, dims, str, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
     }
     dim3 grid((unsigned)nsplit, (unsigned)p.Hkv, (unsigned)p.B);
     const int32_t *bt = paged ? paged->block_table : nullptr;
     const int maxp = paged ? paged->max_pages : 0, psz = paged ? paged->page_size : 0;
     const int npool = paged ? paged->num_pages : 0;
-#define ATF_DEC_TC(DD, PK, PG)                                                                                 \
+#define ATF_DEC_TC_NT(DD, PK, PG, NT)                                                                          \
     do {                                                                                                       \
         const int smem = dtc::Cfg<DD>::Request;                                                                \
-        if ((e = cudaFuncSetAttribute(dtc::decode_tc_kernel<DD, PK, PG>,                                      \
+        if ((e = cudaFuncSetAttribute(dtc::decode_tc_kernel<DD, PK, PG, NT>,                                  \
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)      \
             return e;                                                                                          \
-        dtc::decode_tc_kernel<DD, PK, PG><<<grid, dtc::kThreads, smem, s>>>(                                  \
+        dtc::decode_tc_kernel<DD, PK, PG, NT><<<grid, dtc::kThreads, smem, s>>>(                              \
             tk, tv, q, seqlens, workspace, p.Hq, p.Hkv, nhd, krot, split_keys, nsplit, wp, status, limit_ns,  \
-            bt, maxp, psz, npool);                                                                             \
+            bt, maxp, psz, npool, rows128);                                                                    \
+    } while (0)
+#define ATF_DEC_TC(DD, PK, PG)                                                                                 \
+    do {                                                                                                       \
+        if (p.Hq / p.Hkv <= 8) ATF_DEC_TC_NT(DD, PK, PG, 1);                                                   \
+        else ATF_DEC_TC_NT(DD, PK, PG, 2);                                                                     \
     } while (0)
     if (p.D == 128) {
         if (paged) {
@@ -614,6 +688,7 @@ cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, cons
         }
     }
 #undef ATF_DEC_TC
+#undef ATF_DEC_TC_NT
     return cudaGetLastError();
 }
 
