@@ -180,9 +180,15 @@ __global__ void __launch_bounds__(32 * kDecodeWarps) decode_split_kernel(
 }
 
 // Merge the per-split states (m in log2 units, l, unnormalised acc) of one
-// (sequence, query head) into the output row: block-wide max and weighted sum
-// over the splits, then the accumulators summed by split-parallel thread groups.
-constexpr int kMergeThreads = 256;
+// (sequence, query head) into the output row.  A block takes a slice of
+// kMergeDims output dims: it forms the max and the weighted sum over all splits
+// (block-wide reductions), then kMergeParts thread groups accumulate interleaved
+// splits for its dims and add their parts through shared memory.  The grid
+// (query heads x sequences x dim slices) keeps enough split states in flight to
+// hide memory latency.
+constexpr int kMergeDims = 32;
+constexpr int kMergeParts = 8;
+constexpr int kMergeThreads = kMergeDims * kMergeParts;
 
 __device__ __forceinline__ float block_reduce(float v, bool is_max, float *red) {
 #pragma unroll
@@ -206,7 +212,7 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float *red) 
 __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float *__restrict__ ws, void *out,
                                                                      int out_f32, int Hq, int nsplit, int D) {
     __shared__ float red[32];
-    __shared__ float part_acc[kMergeThreads];
+    __shared__ float part_acc[kMergeParts][kMergeDims];
     const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     const float *base = ws + ((size_t)b * Hq + h) * nsplit * (D + 2);
     float mx = -INFINITY;
@@ -221,23 +227,23 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float
         if (st[1] > 0.f) ls += st[1] * exp2f(st[0] - M);
     }
     const float Lsum = block_reduce(ls, false, red);
-    const int nparts = kMergeThreads / D, part = tid / D, d = tid % D;
+    const int part = tid / kMergeDims, dl = tid % kMergeDims;
+    const int d = blockIdx.z * kMergeDims + dl;
     float a = 0.f;
-    if (part < nparts) {
-#pragma unroll 4
-        for (int s = part; s < nsplit; s += nparts) {
-            const float *st = base + (size_t)s * (D + 2);
-            const float l = st[1];
-            if (l > 0.f) a += st[2 + d] * exp2f(st[0] - M);
-        }
+#pragma unroll 8
+    for (int s = part; s < nsplit; s += kMergeParts) {
+        const float *st = base + (size_t)s * (D + 2);
+        const float l = st[1];
+        if (l > 0.f) a += st[2 + d] * exp2f(st[0] - M);
     }
-    part_acc[tid] = a;
+    part_acc[part][dl] = a;
     __syncthreads();
-    if (tid < D) {
+    if (tid < kMergeDims) {
         float acc = 0.f;
-        for (int pp = 0; pp < nparts; ++pp) acc += part_acc[pp * D + tid];
+#pragma unroll
+        for (int pp = 0; pp < kMergeParts; ++pp) acc += part_acc[pp][tid];
         const float val = acc / Lsum;
-        const size_t o = ((size_t)b * Hq + h) * D + tid;
+        const size_t o = ((size_t)b * Hq + h) * D + d;
         if (out_f32) reinterpret_cast<float *>(out)[o] = val;
         else reinterpret_cast<__nv_bfloat16 *>(out)[o] = __float2bfloat16_rn(val);
     }
@@ -272,8 +278,8 @@ cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const i
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<<<dim3((unsigned)p.Hq, (unsigned)p.B), kMergeThreads, 0, s>>>(workspace, out, out_f32,
-                                                                                        p.Hq, nsplit, p.D);
+    decode_merge_kernel<<<dim3((unsigned)p.Hq, (unsigned)p.B, (unsigned)(p.D / kMergeDims)), kMergeThreads, 0, s>>>(
+        workspace, out, out_f32, p.Hq, nsplit, p.D);
     return cudaGetLastError();
 }
 
