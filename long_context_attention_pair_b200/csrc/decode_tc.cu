@@ -49,7 +49,9 @@ constexpr float kRescaleThreshold = 8.0f;
 
 template <int D>
 struct Cfg {
-    static constexpr int kStages = 3;
+    // Two stages per CTA and three CTAs per SM (74 KB of shared memory each): more
+    // consumer warps to hide latency, as many bytes in flight as three stages at two.
+    static constexpr int kStages = 2;
     static constexpr int H = D / 2;
     static constexpr int C = D / 16;                   // chunks of 8 pairs
     // K stage: packed [c][64 keys][32 B] (SW128 as 16 rows of 128 B, or SW32), natural
@@ -121,15 +123,14 @@ __device__ __forceinline__ void mask_pairs(uint32_t &lo, uint32_t &hi, bool keep
     hi &= m;
 }
 
-// The natural-layout kernel (rotation at load) is asked for two CTAs per SM, which
-// lets the compiler use more registers than its default; the packed kernel keeps
-// the default, which measured faster.
+// Three CTAs per SM for groups of up to 8 heads (160 threads each, at most 128
+// registers per thread); larger groups keep the registers their accumulators need.
 // kPaged: K and V live in pages of page_size tokens (a multiple of the 64-key
 // stage), page block_table[b * max_pages + i] holding keys i*page_size.. of
 // sequence b; the maps index pages along their outermost axis.
 // NT: tiles of 8 query heads (a GQA group of G <= 8 heads takes one tile, up to 16 two).
 template <int D, bool kPacked, bool kPaged, int NT>
-__global__ void __launch_bounds__(kThreads, kPacked ? 0 : 2) decode_tc_kernel(
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const void *q_,
     const int32_t *__restrict__ seqlens, float *__restrict__ ws, int Hq, int Hkv, int nhd, int krot, int split_keys,
     int nsplit, const __grid_constant__ WindowParams wp, int *status, uint64_t limit_ns,
