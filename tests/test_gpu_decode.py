@@ -52,6 +52,9 @@ SMALL = [
     (1, 16, 1, 900, 64, [900], 10.0, 0.25, 0, "bf16"),
     (2, 6, 2, 3000, 128, [3000, 17], 5e5, 16.0, 0, "f32"),
     (1, 4, 2, 1500, 64, [1500], 1e4, 1.0, 1, "f32"),
+    # groups of 9..16 heads take two 8-head tiles of the MMA's N
+    (2, 24, 2, 2100, 128, [2100, 1500], 5e5, 16.0, 0, "bf16"),
+    (1, 10, 1, 1300, 64, [1300], 1e4, 2.0, 1, "bf16"),
 ]
 
 
@@ -74,6 +77,9 @@ def test_decode_matches_oracle(oracle, B, Hq, Hkv, Nmax, D, seqlens, base, kwin,
     (2, 28, 4, 3000, 128, [3000, 2048], 1e7, 16.0),
     (2, 7, 1, 4097, 64, [4097, 300], 1e6, 8.0),
     (1, 16, 1, 900, 64, [900], 10.0, 0.25),
+    # two head tiles at D = 128; a cache length that is not a multiple of 4
+    (2, 24, 2, 2102, 128, [2102, 999], 5e5, 16.0),
+    (1, 12, 1, 2048, 128, [2048], 1e4, 4.0),
 ])
 def test_packed_rotated_cache_matches_oracle(oracle, B, Hq, Hkv, Nmax, D, seqlens, base, kwin):
     # The RoPE pre-pass writes the packed cache from the un-rotated keys; the oracle

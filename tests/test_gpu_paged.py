@@ -53,6 +53,7 @@ CASES = [
     (2, 7, 1, 2048, 64, 256, [2048, 777], 1e6, 8.0, 0),
     (2, 28, 4, 3072, 128, 128, [3072, 3000], 1e7, math.inf, 0),
     (2, 4, 4, 1024, 128, 64, [1024, 65], 1e4, 2.0, 1),
+    (1, 16, 1, 1024, 128, 64, [1000], 1e4, 4.0, 0),
 ]
 
 
