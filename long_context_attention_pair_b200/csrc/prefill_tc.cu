@@ -30,7 +30,10 @@
 //   warp 10          zeroes the fully-pruned pairs of the first loaded K~ chunk
 //                    and stages the tile's boundary pairs as fp32 for the fix-up
 //   warp 11          PV issuer: O_h += P_h V (P from TMEM, V from smem)
-// TMEM columns: O0 [256,256+D), O1 [256+D,256+2D); S and P as in Cfg below.
+// For D = 64 with no pair pruned anywhere the launcher takes the one-head form
+// instead: 8 warps (softmax 0-3, then producer, QK, fix-up, PV), 256 TMEM
+// columns and two K/V stages, so that two CTAs share an SM.
+// TMEM columns: as in Cfg below.
 // Every mbarrier wait is bounded in time; on expiry the CTA records
 // ATFLASH_ERR_TIMEOUT in the device status word, lets its copies land, drains
 // its tensor-core work, frees TMEM and exits.
@@ -46,9 +49,15 @@ namespace tc {
 
 constexpr int kBM = 128;
 constexpr int kBN = 128;
-constexpr int kThreads = 384;
-constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpFix = 10, kWarpPv = 11;
-constexpr uint32_t kTmemCols = 512;
+// NH query heads per CTA (2: one CTA per SM, the heads share every K/V tile; 1:
+// two CTAs per SM, which run out of phase so one CTA's exp2 pass overlaps the
+// other's loads, waits and stores).  Warps: 4*NH softmax, then producer, QK
+// issuer, fix-up and PV issuer.
+template <int NH>
+struct Warps {
+    static constexpr int Threads = 32 * (4 * NH + 4);
+    static constexpr int Producer = 4 * NH, Mma = 4 * NH + 1, Fix = 4 * NH + 2, Pv = 4 * NH + 3;
+};
 constexpr uint32_t kChunkBytes = kBN * 32;  // 128 rows x 16 bf16 (one K-step)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
 // Of every 8 element pairs of a softmax row, this many take exp2 on the FMA
@@ -60,31 +69,35 @@ constexpr int kPolyPairsOf8 = 0;
 // from the K~ chunk.
 constexpr int kMaxStagedPairs = 8;
 
-template <int D>
+template <int D, int NH>
 struct Cfg {
     static constexpr int C = D / 16;                  // K-steps of the QK contraction
-    static constexpr int KS = (D == 64) ? 3 : 2;      // K~ stages
-    static constexpr int VS = (D == 64) ? 3 : 2;      // V stages
+    static constexpr int KS = (D == 64 && NH == 2) ? 3 : 2;  // K~ stages
+    static constexpr int VS = KS;                     // V stages
     static constexpr int QBytes = C * kChunkBytes;    // one query tile
     static constexpr int KBytes = C * kChunkBytes;
     static constexpr int VBytes = (D / 64) * 16384;   // 128 keys x 64 dims x 2 B per group
-    static constexpr int OffQ = 0;                    // two query tiles
-    static constexpr int OffK = OffQ + 2 * QBytes;
+    static constexpr int OffQ = 0;                    // NH query tiles
+    static constexpr int OffK = OffQ + NH * QBytes;
     static constexpr int OffV = OffK + KS * KBytes;
     static constexpr int OffBnd = OffV + VS * VBytes;                 // [KS][kMaxStagedPairs][64] float4
     static constexpr int BndBytes = kMaxStagedPairs * 64 * 16;
     static constexpr int OffCtl = OffBnd + KS * BndBytes;
     static constexpr int Total = OffCtl + 2048;
     static constexpr int Request = Total + 1024;
-    static constexpr uint32_t TmemO0 = 256, TmemO1 = 256 + D;
-    // TMEM: D = 64: S0 [0,128), S1 [128,256), O0, O1 [256,384), P0, P1 [384,512).
-    //       D = 128: one S [0,128) shared by the two heads in turn, P0 [128,192),
-    //                P1 [192,256), O0 [256,384), O1 [384,512).
+    // TMEM, two heads: D = 64: S0 [0,128), S1 [128,256), O0, O1 [256,384), P0, P1 [384,512).
+    //                  D = 128: one S [0,128) shared by the two heads in turn, P0 [128,192),
+    //                  P1 [192,256), O0 [256,384), O1 [384,512).
+    //       one head (D = 64 only): S [0,128), O [128,192), P [192,256) of a 256-column
+    //                  allocation, so that two CTAs share the SM's 512 columns.
     // Either way S_t is free again as soon as softmax t has read it into registers.
+    static_assert(NH == 2 || D == 64, "one head per CTA is laid out for D = 64");
+    static constexpr uint32_t TmemCols = NH == 2 ? 512 : 256;
+    static constexpr uint32_t TmemO0 = NH == 2 ? 256 : 128, TmemO1 = 256 + D;
     static constexpr bool SharedS = (D == 128);
     static constexpr bool Token = false;  // alternate the two heads' exp2 passes (measured slower)
     static constexpr uint32_t TmemS0 = 0, TmemS1 = SharedS ? 0 : 128;
-    static constexpr uint32_t TmemP0 = SharedS ? 128 : 384, TmemP1 = SharedS ? 192 : 448;
+    static constexpr uint32_t TmemP0 = NH == 1 ? 192 : (SharedS ? 128 : 384), TmemP1 = SharedS ? 192 : 448;
 };
 
 template <int KS, int VS>
@@ -162,13 +175,17 @@ __device__ __forceinline__ bool wait_drain(uint64_t *bar, uint32_t parity, uint6
 // kVarlen: the batch is packed along the token axis (q, k, v, out [total][H][D],
 // packed Q~/K~ [H][D/16][total][16]); sequence b holds tokens cu[b]..cu[b+1]-1
 // and N is the longest sequence.  Otherwise q/k/v/out are [B][N][H][D].
-template <int D, bool kVarlen>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, bool kVarlen, int NH>
+__global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ WindowParams wp,
                       void *out, int out_f32, float *lse, int64_t N, int Hq, int Hkv, int *status,
                       uint64_t limit_ns, const int32_t *cu_seqlens, int64_t total) {
-    using F = Cfg<D>;
+    using F = Cfg<D, NH>;
+    using W = Warps<NH>;
+    constexpr int kThreads = W::Threads;
+    constexpr int kWarpProducer = W::Producer, kWarpMma = W::Mma, kWarpFix = W::Fix, kWarpPv = W::Pv;
+    constexpr uint32_t kTmemCols = F::TmemCols;
     constexpr int C = F::C;
     constexpr int H = D / 2;
     constexpr int KS = F::KS, VS = F::VS;
@@ -184,13 +201,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int num_qt = (int)((N + kBM - 1) / kBM);
     const int qt = num_qt - 1 - (int)blockIdx.x;  // longest query tiles first
     const int G = Hq / Hkv;
-    const int pairs_per_group = (G + 1) / 2;
+    const int pairs_per_group = (G + NH - 1) / NH;
     const int b = blockIdx.y / (Hkv * pairs_per_group);
     const int rem = blockIdx.y % (Hkv * pairs_per_group);
     const int kvh = rem / pairs_per_group;
     const int hp = rem % pairs_per_group;
-    const int h0 = kvh * G + 2 * hp;
-    const bool two = (2 * hp + 1) < G;  // a second head of the group shares this CTA
+    const int h0 = kvh * G + NH * hp;
+    const bool two = NH == 2 && (2 * hp + 1) < G;  // a second head of the group shares this CTA
     const int nwg = two ? 2 : 1;
     const int64_t n0 = (int64_t)qt * kBM;
     const int nkt = qt + 1;  // key tiles 0..qt (causal)
@@ -243,10 +260,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int *w = ctl->w;
     WaitCtl wc{&ctl->abort_flag, status, limit_ns, 0};
 
-    // Register split: the launch gives every thread 168 registers (384 x 168 =
-    // 64512).  Warpgroup 2 (producer, fix-up, MMA, idle) drops to 96 and the two
-    // softmax warpgroups rise to 200: 128 x 96 + 256 x 200 = 63488 <= 64512.
-    if (warp >= 8) setmaxnreg_dec<96>();
+    // Register split.  Two heads: the launch gives every thread 168 registers
+    // (384 x 168 = 64512); warpgroup 2 (producer, MMA, fix-up, PV) drops to 96 and
+    // the two softmax warpgroups rise to 200: 128 x 96 + 256 x 200 = 63488 <= 64512.
+    // One head (two CTAs per SM): 128 registers at launch (256 x 128 = 32768);
+    // warpgroup 1 drops to 56 and the softmax warpgroup rises to 200:
+    // 128 x 56 + 128 x 200 = 32768.
+    if constexpr (NH == 2) {
+        if (warp >= 8) setmaxnreg_dec<96>();
+    } else {
+        if (warp >= 4) setmaxnreg_dec<56>();
+    }
     if (warp == kWarpProducer) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -407,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok && lane == 0) umma_commit(&ctl->v_empty[vs]);
             __syncwarp();
         }
-    } else if (warp < 8) {
+    } else if (warp < 4 * NH) {
         // ------------------------------------------------------------- softmax
         setmaxnreg_inc<200>();
         const int t = warp >> 2;  // which head of the pair
@@ -729,22 +753,30 @@ cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *
     }
     const int num_qt = (int)((p.N + tc::kBM - 1) / tc::kBM);
     const int G = p.Hq / p.Hkv;
-    dim3 grid((unsigned)num_qt, (unsigned)(p.B * p.Hkv * ((G + 1) / 2)));
     cudaError_t e;
-#define ATF_PREFILL_TC(DD, VL)                                                                                   \
+#define ATF_PREFILL_TC(DD, VL, NHH)                                                                              \
     do {                                                                                                         \
-        const int smem = tc::Cfg<DD>::Request;                                                                  \
-        e = cudaFuncSetAttribute(tc::prefill_tc_kernel<DD, VL>, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
-                                 smem);                                                                          \
+        const int smem = tc::Cfg<DD, NHH>::Request;                                                             \
+        dim3 grid((unsigned)num_qt, (unsigned)(p.B * p.Hkv * ((G + NHH - 1) / NHH)));                          \
+        e = cudaFuncSetAttribute(tc::prefill_tc_kernel<DD, VL, NHH>,                                            \
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                             \
         if (e != cudaSuccess) return e;                                                                          \
-        tc::prefill_tc_kernel<DD, VL><<<grid, tc::kThreads, smem, s>>>(tq, tk, tv, wp, out, out_f32, lse, p.N,  \
-                                                                       p.Hq, p.Hkv, status, wait_limit_ns,     \
-                                                                       cu_seqlens, total);                     \
+        tc::prefill_tc_kernel<DD, VL, NHH><<<grid, tc::Warps<NHH>::Threads, smem, s>>>(                         \
+            tq, tk, tv, wp, out, out_f32, lse, p.N, p.Hq, p.Hkv, status, wait_limit_ns, cu_seqlens, total);      \
     } while (0)
     if (p.D == 128) {
-        if (varlen) ATF_PREFILL_TC(128, true); else ATF_PREFILL_TC(128, false);
+        if (varlen) ATF_PREFILL_TC(128, true, 2); else ATF_PREFILL_TC(128, false, 2);
     } else if (p.D == 64) {
-        if (varlen) ATF_PREFILL_TC(64, true); else ATF_PREFILL_TC(64, false);
+        // No pair pruned anywhere (k = inf, or windows covering the longest sequence):
+        // one head per CTA, two CTAs per SM measured faster (no boundary work to share
+        // between heads).  With pruning, two heads per CTA share every K~ tile's
+        // zeroing and boundary staging and measured faster.
+        const bool unpruned = (int64_t)wp.w[0] >= p.N - 1;
+        if (unpruned) {
+            if (varlen) ATF_PREFILL_TC(64, true, 1); else ATF_PREFILL_TC(64, false, 1);
+        } else {
+            if (varlen) ATF_PREFILL_TC(64, true, 2); else ATF_PREFILL_TC(64, false, 2);
+        }
     } else {
         return cudaErrorInvalidValue;
     }

@@ -49,6 +49,7 @@ def check_against_oracle(oracle, q, k, v, cu, out, base, kwin, max_rows=48, lse=
     ([700, 1, 0, 257, 2049], 6, 2, 128, 5e5, 16.0),
     ([513, 64, 1500], 7, 1, 128, 1e7, math.inf),
     ([33, 4000], 2, 2, 64, 10.0, 0.25),
+    ([300, 1, 0, 700], 7, 1, 64, 1e4, math.inf),
 ])
 def test_varlen_matches_oracle_per_sequence(oracle, lens, Hq, Hkv, D, base, kwin):
     q, k, v, cu = packed_batch(61, lens, Hq, Hkv, D)
