@@ -83,7 +83,7 @@ KERNELS_PER_STEP = 5  # rope_pack(q), rope_pack(k), prefill_tc, decode_split, de
 # DRAM bytes per launch of the tcgen05 prefill kernel on this workload, from one
 # ncu capture (profiles/prefill_tc_qwen05b_32k.md).  Valid only while the
 # kernel source hashes to `source_sha1`; otherwise the line reports null.
-TRAFFIC = {"bytes_per_launch": 98930944, "source_sha1": "d7bb473dfa1cc9a4b88a7ba8fb42edfb2750ff10"}
+TRAFFIC = {"bytes_per_launch": 99188992, "source_sha1": "67d3d80e1932ab93afb73bd40c88732f7a2d323c"}
 
 
 def parse():
