@@ -477,48 +477,82 @@ def run_decode(args, wl):
 
 
 def e2e(atf, q, k, v, wl, args, dev, world):
-    """Same metric through the public API with host buffers: H2D inputs, prefill,
-    decode of the last row, D2H outputs, all inside the timed region."""
+    """Same metric through the public API with host buffers.  Every step copies
+    its inputs from pinned host memory (H2D q/k/v/seqlens), runs the prefill and
+    the decode of the last row, and reads its outputs back (D2H out and the
+    decoded row), all inside the timed region.  Steps are pipelined over two
+    device buffer sets and three streams (copy in, compute, copy out), as a
+    serving loop would run them: step i's copies overlap step i-1's compute."""
     import torch
     B, N, Hq, Hkv, D = wl["B"], wl["N"], wl["Hq"], wl["Hkv"], wl["D"]
     base, kwin = wl["rope_base"], wl["k_window"]
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     hsl = torch.full((B,), N, dtype=torch.int32).pin_memory()
-    hout = torch.empty((B, N, Hq, D), dtype=torch.bfloat16).pin_memory()
-    hdec = torch.empty((B, Hq, D), dtype=torch.bfloat16).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dsl = torch.empty((B,), dtype=torch.int32, device=dev)
-    dout = torch.empty_like(q)
-    ws = torch.empty(atf.prefill_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device=dev)
-    dws = torch.empty(atf.decode_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
+    nbuf = 2
+    hout = [torch.empty((B, N, Hq, D), dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
+    hdec = [torch.empty((B, Hq, D), dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
+    bufs = []
+    for _ in range(nbuf):
+        bufs.append({
+            "q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
+            "sl": torch.empty((B,), dtype=torch.int32, device=dev), "out": torch.empty_like(q),
+            "qlast": torch.empty((B, Hq, D), dtype=q.dtype, device=dev),
+            "dec": torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev),
+            "ws": torch.empty(atf.prefill_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device=dev),
+            "dws": torch.empty(atf.decode_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device=dev),
+        })
+    s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_done = [ev() for _ in range(nbuf)]
+    comp_done = [ev() for _ in range(nbuf)]
+    out_done = [ev() for _ in range(nbuf)]
+    used = [False] * nbuf
     steps = max(3, args.steps // 10)
 
-    def step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        dsl.copy_(hsl, non_blocking=True)
-        atf.prefill(dq, dk, dv, base, kwin, out=dout, workspace=ws)
-        dec = atf.decode(dq[:, N - 1].contiguous(), dk, dv, dsl, base, kwin, kv_layout="NHD", workspace=dws)
-        hout.copy_(dout, non_blocking=True)
-        hdec.copy_(dec, non_blocking=True)
+    def step(i):
+        bi = i % nbuf
+        d = bufs[bi]
+        with torch.cuda.stream(s_in):
+            if used[bi]:
+                s_in.wait_event(comp_done[bi])  # step i-2 is done reading these inputs
+            d["q"].copy_(hq, non_blocking=True)
+            d["k"].copy_(hk, non_blocking=True)
+            d["v"].copy_(hv, non_blocking=True)
+            d["sl"].copy_(hsl, non_blocking=True)
+            in_done[bi].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(in_done[bi])
+            if used[bi]:
+                s_comp.wait_event(out_done[bi])  # step i-2's outputs have been read back
+            atf.prefill(d["q"], d["k"], d["v"], base, kwin, out=d["out"], workspace=d["ws"], stream=s_comp)
+            d["qlast"].copy_(d["q"][:, N - 1])
+            atf.decode(d["qlast"], d["k"], d["v"], d["sl"], base, kwin, kv_layout="NHD", out=d["dec"],
+                       workspace=d["dws"], stream=s_comp)
+            comp_done[bi].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[bi])
+            hout[bi].copy_(d["out"], non_blocking=True)
+            hdec[bi].copy_(d["dec"], non_blocking=True)
+            out_done[bi].record(s_out)
+        used[bi] = True
 
-    for _ in range(2):
-        step()
+    for i in range(2):
+        step(i)
     barrier(world)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        step()
-    b.record(stream)
+    a.record(s_in)
+    for i in range(steps):
+        step(i)
+    # The last step's read-back ends the timed region; s_out orders it after every step.
+    b.record(s_out)
     torch.cuda.synchronize()
     ms = reduce_max(a.elapsed_time(b), world, dev)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsl))
-    d2h = sum(t.numel() * t.element_size() for t in (hout, hdec))
+    d2h = sum(t.numel() * t.element_size() for t in (hout[0], hdec[0]))
     return {"value": round(world * B * N * steps / (ms / 1e3), 1), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / steps, 4)}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / steps, 4),
+            "pipelined": "2 buffer sets, H2D / compute / D2H streams"}
 
 
 def main():
