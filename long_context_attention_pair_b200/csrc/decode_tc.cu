@@ -24,9 +24,11 @@
 //
 // Packed cache (ATFLASH_KV_PACKED): K already rotated and stored as the RoPE
 // pre-pass writes it, [B*Hkv][D/16][Nmax][16] with 8 frequency pairs per 32-byte
-// chunk.  A pruned chunk of 64 keys is then 2 KB of HBM that is never fetched;
-// in the natural layouts a key's pruned dims are a short prefix of each 128-byte
-// half and HBM's access granularity fetches them anyway.  The 2 KB of one chunk
+// chunk.  A pruned chunk of 64 keys is then 2 KB of HBM that is never fetched.
+// In the natural layouts a key's pruned dims are a prefix of each half-row; the
+// copy fetches each half in 32-byte (16-dim) boxes from the first 32-byte sector
+// that some key of the stage keeps, the finest cut that saves DRAM traffic (the
+// DRAM sector is 32 bytes).  The 2 KB of one chunk
 // of a stage are contiguous, so the copy views them as 16 rows of 128 bytes
 // (4 keys per row, SWIZZLE_128B) rather than 64 rows of 32 bytes: a quarter of
 // the TMA row requests, which bound the producer otherwise.  That view needs
@@ -55,7 +57,7 @@ struct Cfg {
     static constexpr int H = D / 2;
     static constexpr int C = D / 16;                   // chunks of 8 pairs
     // K stage: packed [c][64 keys][32 B] (SW128 as 16 rows of 128 B, or SW32), natural
-    // [D/64][64 keys][64 dims] SW128 like V.
+    // [half][D/32 16-dim groups][64 keys][32 B] SW32.
     static constexpr int KBytes = C * 2 * 1024;
     static constexpr int VBytes = (D / 64) * 8192;     // [D/64][64 keys][64 dims] bf16, SW128
     static constexpr int OffK = 0;
@@ -223,8 +225,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
             }
             __syncwarp();
             if (lane == 0) {
-                // Natural layouts fetch whole K rows (their pruned dims cost DRAM sectors anyway).
-                const uint32_t kbytes = kPacked ? (uint32_t)(C - c_lo) * 2048u : (uint32_t)F::KBytes;
+                // Natural layouts: 16-dim groups g >= g_lo of both halves (32-byte sectors).
+                constexpr int NG = H / 16;  // 16-dim groups per half
+                const int g_lo = c_lo >> 1;
+                const uint32_t kbytes =
+                    kPacked ? (uint32_t)(C - c_lo) * 2048u : (uint32_t)(2 * (NG - g_lo)) * 2048u;
                 const uint32_t bytes = kbytes + (uint32_t)F::VBytes;
                 mbar_expect_tx(&bars->full[st], bytes);
                 uint8_t *kst = sK + st * F::KBytes;
@@ -241,8 +246,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
                         for (int c = c_lo; c < C; ++c)
                             tma_load_3d(kst + c * 2048, &tm_k, &bars->full[st], 0, kk / 4, (page * Hkv + g) * C + c);
                     } else {
-                        for (int gi = 0; gi < D / 64; ++gi)
-                            tma_load_4d(kst + gi * 8192, &tm_k, &bars->full[st], 64 * gi, g, kk, page);
+                        for (int hf = 0; hf < 2; ++hf)
+                            for (int gg = g_lo; gg < NG; ++gg)
+                                tma_load_4d(kst + (hf * NG + gg) * 2048, &tm_k, &bars->full[st], hf * H + 16 * gg, g,
+                                            kk, page);
                     }
                     for (int gi = 0; gi < D / 64; ++gi)
                         tma_load_4d(sV + st * F::VBytes + gi * 8192, &tm_v, &bars->full[st], 64 * gi, g, kk, page);
@@ -251,12 +258,14 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
                     for (int c = c_lo; c < C; ++c)
                         tma_load_3d(kst + c * 2048, &tm_k, &bars->full[st], 0, ky, (b * Hkv + g) * C + c);
                 } else {
-                    // 64 keys x 64 dims per box, SWIZZLE_128B, like V.
-                    for (int gi = 0; gi < D / 64; ++gi) {
-                        uint8_t *dst = kst + gi * 8192;
-                        if (nhd) tma_load_4d(dst, &tm_k, &bars->full[st], 64 * gi, g, (int)k0, b);
-                        else tma_load_3d(dst, &tm_k, &bars->full[st], 64 * gi, (int)k0, b * Hkv + g);
-                    }
+                    // 64 keys x 16 dims per box, SWIZZLE_32B.
+                    for (int hf = 0; hf < 2; ++hf)
+                        for (int gg = g_lo; gg < NG; ++gg) {
+                            uint8_t *dst = kst + (hf * NG + gg) * 2048;
+                            const int x = hf * H + 16 * gg;
+                            if (nhd) tma_load_4d(dst, &tm_k, &bars->full[st], x, g, (int)k0, b);
+                            else tma_load_3d(dst, &tm_k, &bars->full[st], x, (int)k0, b * Hkv + g);
+                        }
                 }
                 if constexpr (!kPaged) {
                     for (int gi = 0; gi < D / 64; ++gi) {
@@ -398,12 +407,12 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
                         if (c < (c_warp > c_stage ? c_warp : c_stage)) continue;
                         const bool masked = c < c_keep;
                         uint32_t b0, b1, b2, b3;
-                        // Rows of 64 dims (128 B, SWIZZLE_128B: 16-byte unit ^= key & 7); matrix
-                        // mi: keys +8*(mi>>1), dims (mi&1)*H + 8c .. +8 of each key.
+                        // 16-dim groups of 64 keys x 32 B (SWIZZLE_32B: 16-byte unit ^= key bit 2);
+                        // matrix mi: keys +8*(mi>>1), dims (mi&1)*H + 8c .. +8 of each key, i.e.
+                        // unit c&1 of group c>>1 of half mi&1.
                         const int key = 16 * wq + 8 * (mi >> 1) + ri;
-                        const int dim0 = (mi & 1) * H + 8 * c;
-                        const uint32_t addr =
-                            kst + (dim0 >> 6) * 8192 + key * 128 + ((((dim0 & 63) >> 3) ^ (key & 7)) << 4);
+                        const uint32_t addr = kst + ((mi & 1) * (H / 16) + (c >> 1)) * 2048 + key * 32 +
+                                              ((((uint32_t)c & 1u) ^ (((uint32_t)key >> 2) & 1u)) << 4);
                         ldsm_x4(addr, b0, b1, b2, b3);
                         const int p0 = 8 * c + 2 * tq, p1 = p0 + 1;
                         const int w0 = sw[p0], w1 = sw[p1];
@@ -624,7 +633,8 @@ cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, cons
             cuuint32_t boxk[3] = {64, dtc::kStageKeys / 4, 1};
             if ((e = make_map_bf16(&tk, kc, 3, dk, sk, boxk, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
         } else {
-            if ((e = make_map_bf16(&tk, kc, 4, dv, sv, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
+            cuuint32_t boxk[4] = {16, 1, dtc::kStageKeys, 1};
+            if ((e = make_map_bf16(&tk, kc, 4, dv, sv, boxk, CU_TENSOR_MAP_SWIZZLE_32B)) != cudaSuccess) return e;
         }
     } else if (packed) {
         // K: [B*Hkv*D/16][Nmax][16] packed chunks; V: [B][Hkv][Nmax][D].
@@ -646,14 +656,14 @@ cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, cons
     } else if (nhd) {
         cuuint64_t dims[4] = {Dd, Hk, Nm, Bb};
         cuuint64_t str[3] = {Dd * 2, Hk * Dd * 2, Nm * Hk * Dd * 2};
-        cuuint32_t boxv[4] = {64, 1, dtc::kStageKeys, 1};
-        if ((e = make_map_bf16(&tk, kc, 4, dims, str, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
+        cuuint32_t boxk[4] = {16, 1, dtc::kStageKeys, 1}, boxv[4] = {64, 1, dtc::kStageKeys, 1};
+        if ((e = make_map_bf16(&tk, kc, 4, dims, str, boxk, CU_TENSOR_MAP_SWIZZLE_32B)) != cudaSuccess) return e;
         if ((e = make_map_bf16(&tv, vc, 4, dims, str, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
     } else {
         cuuint64_t dims[3] = {Dd, Nm, Bb * Hk};
         cuuint64_t str[2] = {Dd * 2, Nm * Dd * 2};
-        cuuint32_t boxv[3] = {64, dtc::kStageKeys, 1};
-        if ((e = make_map_bf16(&tk, kc, 3, dims, str, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
+        cuuint32_t boxk[3] = {16, dtc::kStageKeys, 1}, boxv[3] = {64, dtc::kStageKeys, 1};
+        if ((e = make_map_bf16(&tk, kc, 3, dims, str, boxk, CU_TENSOR_MAP_SWIZZLE_32B)) != cudaSuccess) return e;
         if ((e = make_map_bf16(&tv, vc, 3, dims, str, boxv, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
     }
     dim3 grid((unsigned)nsplit, (unsigned)p.Hkv, (unsigned)p.B);
