@@ -84,6 +84,12 @@ KERNELS_PER_STEP = 5  # rope_pack(q), rope_pack(k), prefill_tc, decode_split, de
 # ncu capture (profiles/prefill_tc_qwen05b_32k.md).  Valid only while the
 # kernel source hashes to `source_sha1`; otherwise the line reports null.
 TRAFFIC = {"bytes_per_launch": 99188992, "source_sha1": "67d3d80e1932ab93afb73bd40c88732f7a2d323c"}
+# DRAM bytes per launch of the decode kernel (split states included, merge not) on
+# the full-size workload, from one single-pass ncu capture
+# (profiles/decode_tc_qwen7b_packed_4x128k.md); valid while decode_tc.cu hashes to
+# `source_sha1`.
+DECODE_TRAFFIC = {"decode_1m_packed": {"bytes_per_launch": 6607551744,
+                                       "source_sha1": "50f3c0bd54c58fcc6df42a9e4367cf7639e852af"}}
 
 
 def parse():
@@ -110,13 +116,21 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_sha1():
-    path = os.path.join(ROOT, "long_context_attention_pair_b200", "csrc", "prefill_tc.cu")
+def kernel_sha1(name="prefill_tc.cu"):
+    path = os.path.join(ROOT, "long_context_attention_pair_b200", "csrc", name)
     with open(path, "rb") as f:
         return hashlib.sha1(f.read()).hexdigest()
 
 
 # ---------------------------------------------------------------- distributed
+def decode_traffic(workload, L):
+    """Captured DRAM bytes of one decode launch for this workload, or None."""
+    rec = DECODE_TRAFFIC.get(workload)
+    if rec is None or L != DECODE_WORKLOADS[workload]["N"] or rec["source_sha1"] != kernel_sha1("decode_tc.cu"):
+        return None
+    return rec["bytes_per_launch"]
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -467,7 +481,7 @@ def run_decode(args, wl):
             "config": dict(wl, l2="inputs larger than L2 (cache of %.1f GB)" % (2 * B * Hkv * L * D * 2 / 1e9)),
             "decode": {"us_per_call": round(1e3 * ms, 2), "us_per_token": round(1e3 * ms / B, 2)},
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": decode_traffic(args.workload, L),
                          "kernel": f"decode_tc_kernel<{D}> + decode_merge_kernel",
                          "bytes_per_call": nbytes, "peak_source": src},
             "window_off": {"ms_per_step": round(ms_off, 4), "us_per_token": round(1e3 * ms_off / B, 2)},
