@@ -89,7 +89,7 @@ TRAFFIC = {"bytes_per_launch": 99188992, "source_sha1": "67d3d80e1932ab93afb73bd
 # (profiles/decode_tc_qwen7b_packed_4x128k.md); valid while decode_tc.cu hashes to
 # `source_sha1`.
 DECODE_TRAFFIC = {"decode_1m_packed": {"bytes_per_launch": 6607551744,
-                                       "source_sha1": "50f3c0bd54c58fcc6df42a9e4367cf7639e852af"}}
+                                       "source_sha1": "60819fd860ef68921aa18d358fbc1c8b40b9508a"}}
 
 
 def parse():

@@ -235,6 +235,33 @@ int atflash_decode(const void *q, const void *kcache, const void *vcache, const 
                    void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Scaled RoPE: the calls below take the per-pair frequencies theta_r as a HOST
+ * table of D/2 fp64 values instead of a base, for models whose configuration
+ * rescales the RoPE frequencies ("Porting to something else" derives the window
+ * table from the model's RoPE configuration, rope_scaling included).  Both the
+ * rotation (angle position * theta_r) and the window (w_r = floor(k * 2*pi /
+ * theta_r)) use the table.  The table must be finite, in (0, pi], and
+ * non-increasing in r (so that the pairs kept at any distance are a suffix of
+ * the pairs); otherwise ATFLASH_ERR_INVALID_ARG.  The library reads the table
+ * during the call only.  Every other argument, layout and error is that of the
+ * base-taking call of the same name; a table equal to atflash_theta_table's
+ * gives bit-identical results to that call.
+ */
+/* theta_out (HOST, D/2 fp64) = base^(-2r/D), the table the base-taking calls use. */
+int atflash_theta_table(int D, double rope_base, double *theta_out);
+int atflash_window_table_theta(int D, const double *theta, double k_window, int64_t N, int64_t *w_out);
+int atflash_pruned_terms_theta(int64_t N, int D, const double *theta, double k_window, atflash_terms *out);
+int atflash_rope_pack_theta(const void *x, void *y, int B, int64_t N, int H, int D, const double *theta,
+                            int in_dtype, cudaStream_t stream);
+int atflash_prefill_theta(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
+                          int64_t N, int D, const double *theta, double k_window, int in_dtype, int out_dtype,
+                          float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+int atflash_decode_theta(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens,
+                         void *out, int B, int Hq, int Hkv, int64_t Nmax, int D, const double *theta,
+                         double k_window, int kcache_rotated, int kv_layout, int in_dtype, int out_dtype,
+                         void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Decode that allocates nothing (no counterpart in the paper; an addition of
  * this library).  For callers that cannot allocate device memory at the call
  * site, e.g. a serving loop that must never enter the CUDA allocator once it

@@ -18,7 +18,7 @@ import os
 __all__ = [
     "lib", "prefill", "decode", "pruned_terms", "window_table", "prefill_workspace_bytes",
     "decode_workspace_bytes", "device_status", "AtflashError", "F32", "BF16", "rope_pack", "prefill_packed",
-    "prefill_bf16",
+    "prefill_bf16", "theta_table",
 ]
 
 F32 = 0
@@ -75,9 +75,18 @@ def lib():
         L.atflash_prefill_varlen_workspace_bytes.argtypes = [i, i, i64, i]
         L.atflash_prefill_varlen_workspace_bytes.restype = sz
         L.atflash_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, d, d, i, i, i, vp, sz, vp]
+        dp = ctypes.POINTER(ctypes.c_double)
+        L.atflash_theta_table.argtypes = [i, d, dp]
+        L.atflash_window_table_theta.argtypes = [i, dp, d, i64, ctypes.POINTER(ctypes.c_int64)]
+        L.atflash_pruned_terms_theta.argtypes = [i64, i, dp, d, ctypes.POINTER(Terms)]
+        L.atflash_rope_pack_theta.argtypes = [vp, vp, i, i64, i, i, dp, i, vp]
+        L.atflash_prefill_theta.argtypes = [vp, vp, vp, vp, i, i, i, i64, i, dp, d, i, i, vp, vp, sz, vp]
+        L.atflash_decode_theta.argtypes = [vp, vp, vp, vp, vp, i, i, i, i64, i, dp, d, i, i, i, i, vp, sz, vp]
         for f in ("atflash_window_table", "atflash_pruned_terms", "atflash_prefill", "atflash_prefill_ex",
                   "atflash_decode", "atflash_device_status", "atflash_rope_pack", "atflash_prefill_packed",
-                  "atflash_prefill_varlen", "atflash_decode_paged"):
+                  "atflash_prefill_varlen", "atflash_decode_paged", "atflash_theta_table",
+                  "atflash_window_table_theta", "atflash_pruned_terms_theta", "atflash_rope_pack_theta",
+                  "atflash_prefill_theta", "atflash_decode_theta"):
             getattr(L, f).restype = i
         _lib = L
     return _lib
@@ -92,17 +101,41 @@ def _check(status, what):
         raise AtflashError(status, what)
 
 
-def window_table(D: int, rope_base: float, k_window: float, N: int):
-    """Per-pair windows min(floor(k * lambda_r), N - 1), r < D/2 (host computation)."""
-    arr = (ctypes.c_int64 * (D // 2))()
-    _check(lib().atflash_window_table(D, rope_base, k_window, N, arr), "atflash_window_table")
+def _theta_arg(theta, D):
+    """A caller's RoPE frequency table (scaled RoPE) as a host fp64 array of D/2."""
+    vals = [float(x) for x in theta]
+    if len(vals) != D // 2:
+        raise ValueError(f"theta must hold D/2 = {D // 2} frequencies, got {len(vals)}")
+    return (ctypes.c_double * len(vals))(*vals)
+
+
+def theta_table(D: int, rope_base: float):
+    """theta_r = base^(-2r/D), r < D/2: the frequencies the base-taking calls use."""
+    arr = (ctypes.c_double * (D // 2))()
+    _check(lib().atflash_theta_table(D, float(rope_base), arr), "atflash_theta_table")
     return list(arr)
 
 
-def pruned_terms(N: int, D: int, rope_base: float, k_window: float) -> dict:
+def window_table(D: int, rope_base: float, k_window: float, N: int, *, theta=None):
+    """Per-pair windows min(floor(k * lambda_r), N - 1), r < D/2 (host computation).
+    ``theta`` (D/2 frequencies) replaces base^(-2r/D) for scaled RoPE."""
+    arr = (ctypes.c_int64 * (D // 2))()
+    if theta is None:
+        _check(lib().atflash_window_table(D, rope_base, k_window, N, arr), "atflash_window_table")
+    else:
+        _check(lib().atflash_window_table_theta(D, _theta_arg(theta, D), k_window, N, arr),
+               "atflash_window_table_theta")
+    return list(arr)
+
+
+def pruned_terms(N: int, D: int, rope_base: float, k_window: float, *, theta=None) -> dict:
     """Closed-form kept/pruned term counts of one (sequence, head)."""
     t = Terms()
-    _check(lib().atflash_pruned_terms(N, D, rope_base, k_window, ctypes.byref(t)), "atflash_pruned_terms")
+    if theta is None:
+        _check(lib().atflash_pruned_terms(N, D, rope_base, k_window, ctypes.byref(t)), "atflash_pruned_terms")
+    else:
+        _check(lib().atflash_pruned_terms_theta(N, D, _theta_arg(theta, D), k_window, ctypes.byref(t)),
+               "atflash_pruned_terms_theta")
     return {"total": t.total, "kept": t.kept, "pruned": t.pruned, "total_dims": t.total_dims,
             "kept_dims": t.kept_dims}
 
@@ -144,12 +177,13 @@ def _dev(t, name):
 
 
 def prefill(q, k, v, rope_base: float, k_window: float = math.inf, *, out=None, out_dtype=None,
-            return_lse: bool = False, workspace=None, stream=None):
+            return_lse: bool = False, workspace=None, stream=None, theta=None):
     """Windowed causal RoPE prefill.
 
     q [B, N, Hq, D], k/v [B, N, Hkv, D] (un-rotated q/k; bf16 -> tensor-core path,
     fp32 -> exact CUDA-core path).  Returns out [B, N, Hq, D] (dtype ``out_dtype``,
-    default q's dtype) and, with ``return_lse``, lse [B, Hq, N] fp32.
+    default q's dtype) and, with ``return_lse``, lse [B, Hq, N] fp32.  ``theta``
+    (D/2 frequencies) replaces base^(-2r/D) for scaled RoPE.
     """
     torch = _torch()
     B, N, Hq, D = q.shape
@@ -164,11 +198,14 @@ def prefill(q, k, v, rope_base: float, k_window: float = math.inf, *, out=None, 
     need = prefill_workspace_bytes(B, Hq, Hkv, N, D, in_dtype)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    st = lib().atflash_prefill_ex(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), B, Hq, Hkv, N, D,
-                                  float(rope_base), float(k_window), in_dtype, _dtype_code(out),
-                                  _dev(lse, "lse") if lse is not None else None, _dev(workspace, "workspace"),
-                                  need, _stream_ptr(stream))
-    _check(st, "atflash_prefill_ex")
+    fn, name = lib().atflash_prefill_ex, "atflash_prefill_ex"
+    rope = float(rope_base)
+    if theta is not None:
+        fn, name, rope = lib().atflash_prefill_theta, "atflash_prefill_theta", _theta_arg(theta, D)
+    st = fn(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), B, Hq, Hkv, N, D, rope, float(k_window),
+            in_dtype, _dtype_code(out), _dev(lse, "lse") if lse is not None else None, _dev(workspace, "workspace"),
+            need, _stream_ptr(stream))
+    _check(st, name)
     return (out, lse) if return_lse else out
 
 
@@ -233,7 +270,7 @@ def decode_paged(q, kpages, vpages, block_table, seqlens, page_size: int, rope_b
     return out
 
 
-def rope_pack(x, rope_base: float, *, out=None, stream=None):
+def rope_pack(x, rope_base: float, *, out=None, stream=None, theta=None):
     """Rotate x [B, N, H, D] once into the packed layout ``prefill_packed`` reads.
 
     bf16 -> [B*H, D/16, N, 16] bf16 (8 pairs per 32-byte chunk, pair-interleaved);
@@ -248,8 +285,12 @@ def rope_pack(x, rope_base: float, *, out=None, stream=None):
     if out is None:
         shape = (B * H, D // 16, N, 16) if dt == BF16 else (B * H, N, D)
         out = torch.empty(shape, dtype=x.dtype, device=x.device)
-    _check(lib().atflash_rope_pack(_dev(x, "x"), _dev(out, "out"), B, N, H, D, float(rope_base), dt,
-                                   _stream_ptr(stream)), "atflash_rope_pack")
+    if theta is None:
+        _check(lib().atflash_rope_pack(_dev(x, "x"), _dev(out, "out"), B, N, H, D, float(rope_base), dt,
+                                       _stream_ptr(stream)), "atflash_rope_pack")
+    else:
+        _check(lib().atflash_rope_pack_theta(_dev(x, "x"), _dev(out, "out"), B, N, H, D, _theta_arg(theta, D), dt,
+                                             _stream_ptr(stream)), "atflash_rope_pack_theta")
     return out
 
 
@@ -282,7 +323,7 @@ def prefill_bf16(q, k, v, out, rope_base: float, k_window: float = math.inf, str
 
 def decode(q, k_cache, v_cache, seqlens, rope_base: float, k_window: float = math.inf, *,
            kcache_rotated: bool = False, kv_layout: str = "HND", out=None, out_dtype=None, workspace=None,
-           stream=None):
+           stream=None, theta=None):
     """Windowed decode: q [B, Hq, D], seqlens int32 [B] (device), caches in
     ``kv_layout`` "HND" [B, Hkv, Nmax, D], "NHD" [B, Nmax, Hkv, D], or "PACKED":
     k_cache = ``rope_pack`` output [B*Hkv, D/16, Nmax, 16] (rotated; requires
@@ -312,11 +353,14 @@ def decode(q, k_cache, v_cache, seqlens, rope_base: float, k_window: float = mat
     need = decode_workspace_bytes(B, Hq, Hkv, Nmax, D)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    st = lib().atflash_decode(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-                              _dev(seqlens, "seqlens"), _dev(out, "out"), B, Hq, Hkv, Nmax, D, float(rope_base),
-                              float(k_window), int(bool(kcache_rotated)), lay, in_dtype, _dtype_code(out),
-                              _dev(workspace, "workspace"), need, _stream_ptr(stream))
-    _check(st, "atflash_decode")
+    fn, name = lib().atflash_decode, "atflash_decode"
+    rope = float(rope_base)
+    if theta is not None:
+        fn, name, rope = lib().atflash_decode_theta, "atflash_decode_theta", _theta_arg(theta, D)
+    st = fn(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(seqlens, "seqlens"),
+            _dev(out, "out"), B, Hq, Hkv, Nmax, D, rope, float(k_window), int(bool(kcache_rotated)), lay, in_dtype,
+            _dtype_code(out), _dev(workspace, "workspace"), need, _stream_ptr(stream))
+    _check(st, name)
     return out
 
 

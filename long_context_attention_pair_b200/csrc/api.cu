@@ -101,15 +101,30 @@ static int check_shape(int B, int Hq, int Hkv, int64_t N) {
     return ATFLASH_OK;
 }
 
-static int fill_window(WindowParams &wp, int D, double base, double k, int64_t N) {
+static int check_theta_args(int D, const double *theta, double k) {
+    if (!theta_valid(D, theta) || isnan(k) || k < 0.0) return ATFLASH_ERR_INVALID_ARG;
+    return ATFLASH_OK;
+}
+
+static int fill_window_theta(WindowParams &wp, int D, const double *theta, double k, int64_t N) {
     int64_t w[kMaxPairs];
-    int rc = window_table(D, base, k, N, w);
+    int rc = window_table_theta(D, theta, k, N, w);
     if (rc != ATFLASH_OK) return rc;
     memset(&wp, 0, sizeof(wp));
     wp.H = D / 2;
-    for (int r = 0; r < D / 2; ++r) wp.w[r] = (int32_t)w[r];  // <= N-1 <= INT32_MAX
-    theta_table(D, base, wp.theta);
+    for (int r = 0; r < D / 2; ++r) {
+        wp.w[r] = (int32_t)w[r];  // <= N-1 <= INT32_MAX
+        wp.theta[r] = theta[r];
+    }
     return ATFLASH_OK;
+}
+
+static int fill_window(WindowParams &wp, int D, double base, double k, int64_t N) {
+    int rc = check_window_args(D, base, k);
+    if (rc != ATFLASH_OK) return rc;
+    double theta[kMaxPairs];
+    theta_table(D, base, theta);
+    return fill_window_theta(wp, D, theta, k, N);
 }
 
 static size_t prefill_ws(int B, int Hq, int Hkv, int64_t N, int D, int in_dtype) {
@@ -147,17 +162,34 @@ int atflash_pruned_terms(int64_t N, int D, double rope_base, double k_window, at
     return pruned_terms(N, D, rope_base, k_window, out);
 }
 
+int atflash_theta_table(int D, double rope_base, double *theta_out) {
+    if (!theta_out) return ATFLASH_ERR_INVALID_ARG;
+    int rc = check_window_args(D, rope_base, 0.0);
+    if (rc != ATFLASH_OK) return rc;
+    theta_table(D, rope_base, theta_out);
+    return ATFLASH_OK;
+}
+
+int atflash_window_table_theta(int D, const double *theta, double k_window, int64_t N, int64_t *w_out) {
+    if (!w_out) return ATFLASH_ERR_INVALID_ARG;
+    return window_table_theta(D, theta, k_window, N, w_out);
+}
+
+int atflash_pruned_terms_theta(int64_t N, int D, const double *theta, double k_window, atflash_terms *out) {
+    return pruned_terms_theta(N, D, theta, k_window, out);
+}
+
 size_t atflash_prefill_workspace_bytes(int B, int Hq, int Hkv, int64_t N, int D, int in_dtype) {
     if (check_shape(B, Hq, Hkv, N) != ATFLASH_OK || D < 2 || D > 2 * kMaxPairs || (D & 1)) return 0;
     if (in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) return 0;
     return prefill_ws(B, Hq, Hkv, N, D, in_dtype);
 }
 
-static int check_prefill_common(int B, int Hq, int Hkv, int64_t N, int D, double base, double k, int in_dtype,
-                                int out_dtype) {
+static int check_prefill_common(int B, int Hq, int Hkv, int64_t N, int D, const double *theta, double k,
+                                int in_dtype, int out_dtype) {
     int rc = check_shape(B, Hq, Hkv, N);
     if (rc != ATFLASH_OK) return rc;
-    if ((rc = check_window_args(D, base, k)) != ATFLASH_OK) return rc;
+    if ((rc = check_theta_args(D, theta, k)) != ATFLASH_OK) return rc;
     if ((in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) ||
         (out_dtype != ATFLASH_F32 && out_dtype != ATFLASH_BF16))
         return ATFLASH_ERR_UNSUPPORTED;
@@ -166,10 +198,10 @@ static int check_prefill_common(int B, int Hq, int Hkv, int64_t N, int D, double
 }
 
 static int run_prefill_packed(const void *qt, const void *kt, const void *v, void *out, int B, int Hq, int Hkv,
-                              int64_t N, int D, double base, double k, int in_dtype, int out_dtype, float *lse,
-                              cudaStream_t stream) {
+                              int64_t N, int D, const double *theta, double k, int in_dtype, int out_dtype,
+                              float *lse, cudaStream_t stream) {
     WindowParams wp;
-    int rc = fill_window(wp, D, base, k, N);
+    int rc = fill_window_theta(wp, D, theta, k, N);
     if (rc != ATFLASH_OK) return rc;
     Problem p{B, Hq, Hkv, D, N};
     const int out_f32 = (out_dtype == ATFLASH_F32);
@@ -185,12 +217,12 @@ static int run_prefill_packed(const void *qt, const void *kt, const void *v, voi
     return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
 }
 
-static int run_rope_pack(const void *x, void *y, int B, int64_t N, int H, int D, double base, int in_dtype,
-                         cudaStream_t stream) {
+static int run_rope_pack(const void *x, void *y, int B, int64_t N, int H, int D, const double *theta,
+                         int in_dtype, cudaStream_t stream) {
     WindowParams wp;
     memset(&wp, 0, sizeof(wp));
     wp.H = D / 2;
-    theta_table(D, base, wp.theta);
+    for (int r = 0; r < D / 2; ++r) wp.theta[r] = theta[r];
     cudaError_t e = (in_dtype == ATFLASH_BF16) ? launch_rope_pack_bf16(x, y, B, N, H, D, wp, stream)
                                                : launch_rope_pack_f32(x, y, B, N, H, D, wp, stream);
     return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
@@ -203,36 +235,59 @@ size_t atflash_rope_pack_bytes(int B, int64_t N, int H, int D, int in_dtype) {
     return 0;
 }
 
-int atflash_rope_pack(const void *x, void *y, int B, int64_t N, int H, int D, double rope_base, int in_dtype,
-                      cudaStream_t stream) {
+static int rope_pack_impl(const void *x, void *y, int B, int64_t N, int H, int D, const double *theta,
+                          int in_dtype, cudaStream_t stream) {
     if (!x || !y) return ATFLASH_ERR_INVALID_ARG;
     int rc = check_shape(B, H, H, N);
     if (rc != ATFLASH_OK) return rc;
-    if ((rc = check_window_args(D, rope_base, 0.0)) != ATFLASH_OK) return rc;
+    if ((rc = check_theta_args(D, theta, 0.0)) != ATFLASH_OK) return rc;
     if (in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) return ATFLASH_ERR_UNSUPPORTED;
     if (in_dtype == ATFLASH_BF16 && D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
     if (!aligned16(x) || (reinterpret_cast<uintptr_t>(y) & 255u)) return ATFLASH_ERR_ALIGNMENT;
-    return run_rope_pack(x, y, B, N, H, D, rope_base, in_dtype, stream);
+    return run_rope_pack(x, y, B, N, H, D, theta, in_dtype, stream);
+}
+
+// theta_r = base^(-2r/D) for the calls that take a RoPE base (validated first).
+struct BaseTheta {
+    double theta[kMaxPairs];
+    int rc;
+    BaseTheta(int D, double base) : rc(check_window_args(D, base, 0.0)) {
+        if (rc == ATFLASH_OK) theta_table(D, base, theta);
+    }
+};
+
+int atflash_rope_pack(const void *x, void *y, int B, int64_t N, int H, int D, double rope_base, int in_dtype,
+                      cudaStream_t stream) {
+    BaseTheta bt(D, rope_base);
+    if (bt.rc != ATFLASH_OK) return bt.rc;
+    return rope_pack_impl(x, y, B, N, H, D, bt.theta, in_dtype, stream);
+}
+
+int atflash_rope_pack_theta(const void *x, void *y, int B, int64_t N, int H, int D, const double *theta,
+                            int in_dtype, cudaStream_t stream) {
+    return rope_pack_impl(x, y, B, N, H, D, theta, in_dtype, stream);
 }
 
 int atflash_prefill_packed(const void *qpack, const void *kpack, const void *v, void *out, int B, int Hq,
                            int Hkv, int64_t N, int D, double rope_base, double k_window, int in_dtype,
                            int out_dtype, float *lse, cudaStream_t stream) {
     if (!qpack || !kpack || !v || !out) return ATFLASH_ERR_INVALID_ARG;
-    int rc = check_prefill_common(B, Hq, Hkv, N, D, rope_base, k_window, in_dtype, out_dtype);
+    BaseTheta bt(D, rope_base);
+    if (bt.rc != ATFLASH_OK) return bt.rc;
+    int rc = check_prefill_common(B, Hq, Hkv, N, D, bt.theta, k_window, in_dtype, out_dtype);
     if (rc != ATFLASH_OK) return rc;
     if ((reinterpret_cast<uintptr_t>(qpack) & 255u) || (reinterpret_cast<uintptr_t>(kpack) & 255u) ||
         !aligned16(v) || !aligned16(out))
         return ATFLASH_ERR_ALIGNMENT;
-    return run_prefill_packed(qpack, kpack, v, out, B, Hq, Hkv, N, D, rope_base, k_window, in_dtype, out_dtype,
+    return run_prefill_packed(qpack, kpack, v, out, B, Hq, Hkv, N, D, bt.theta, k_window, in_dtype, out_dtype,
                               lse, stream);
 }
 
-int atflash_prefill_ex(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
-                       int64_t N, int D, double rope_base, double k_window, int in_dtype, int out_dtype,
-                       float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+static int prefill_ex_impl(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
+                           int64_t N, int D, const double *theta, double k_window, int in_dtype, int out_dtype,
+                           float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
     if (!q || !k || !v || !out) return ATFLASH_ERR_INVALID_ARG;
-    int rc = check_prefill_common(B, Hq, Hkv, N, D, rope_base, k_window, in_dtype, out_dtype);
+    int rc = check_prefill_common(B, Hq, Hkv, N, D, theta, k_window, in_dtype, out_dtype);
     if (rc != ATFLASH_OK) return rc;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATFLASH_ERR_ALIGNMENT;
     const size_t need = prefill_ws(B, Hq, Hkv, N, D, in_dtype);
@@ -242,10 +297,26 @@ int atflash_prefill_ex(const void *q, const void *k, const void *v, void *out, i
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     void *qt = ws;
     void *kt = ws + align256((size_t)B * Hq * N * D * es);
-    if ((rc = run_rope_pack(q, qt, B, N, Hq, D, rope_base, in_dtype, stream)) != ATFLASH_OK) return rc;
-    if ((rc = run_rope_pack(k, kt, B, N, Hkv, D, rope_base, in_dtype, stream)) != ATFLASH_OK) return rc;
-    return run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, rope_base, k_window, in_dtype, out_dtype, lse,
-                              stream);
+    if ((rc = run_rope_pack(q, qt, B, N, Hq, D, theta, in_dtype, stream)) != ATFLASH_OK) return rc;
+    if ((rc = run_rope_pack(k, kt, B, N, Hkv, D, theta, in_dtype, stream)) != ATFLASH_OK) return rc;
+    return run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, theta, k_window, in_dtype, out_dtype, lse, stream);
+}
+
+int atflash_prefill_ex(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
+                       int64_t N, int D, double rope_base, double k_window, int in_dtype, int out_dtype,
+                       float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (!q || !k || !v || !out) return ATFLASH_ERR_INVALID_ARG;
+    BaseTheta bt(D, rope_base);
+    if (bt.rc != ATFLASH_OK) return bt.rc;
+    return prefill_ex_impl(q, k, v, out, B, Hq, Hkv, N, D, bt.theta, k_window, in_dtype, out_dtype, lse, workspace,
+                           workspace_bytes, stream);
+}
+
+int atflash_prefill_theta(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
+                          int64_t N, int D, const double *theta, double k_window, int in_dtype, int out_dtype,
+                          float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return prefill_ex_impl(q, k, v, out, B, Hq, Hkv, N, D, theta, k_window, in_dtype, out_dtype, lse, workspace,
+                           workspace_bytes, stream);
 }
 
 int atflash_prefill(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv, int64_t N,
@@ -358,14 +429,14 @@ int atflash_decode_paged(const void *q, const void *kpages, const void *vpages, 
     return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
 }
 
-int atflash_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out,
-                   int B, int Hq, int Hkv, int64_t Nmax, int D, double rope_base, double k_window,
-                   int kcache_rotated, int kv_layout, int in_dtype, int out_dtype, void *workspace,
-                   size_t workspace_bytes, cudaStream_t stream) {
+static int decode_impl(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out,
+                       int B, int Hq, int Hkv, int64_t Nmax, int D, const double *theta, double k_window,
+                       int kcache_rotated, int kv_layout, int in_dtype, int out_dtype, void *workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
     if (!q || !kcache || !vcache || !seqlens || !out) return ATFLASH_ERR_INVALID_ARG;
     int rc = check_shape(B, Hq, Hkv, Nmax);
     if (rc != ATFLASH_OK) return rc;
-    if ((rc = check_window_args(D, rope_base, k_window)) != ATFLASH_OK) return rc;
+    if ((rc = check_theta_args(D, theta, k_window)) != ATFLASH_OK) return rc;
     if (kcache_rotated != 0 && kcache_rotated != 1) return ATFLASH_ERR_INVALID_ARG;
     if (kv_layout != ATFLASH_KV_HND && kv_layout != ATFLASH_KV_NHD && kv_layout != ATFLASH_KV_PACKED)
         return ATFLASH_ERR_INVALID_ARG;
@@ -382,12 +453,31 @@ int atflash_decode(const void *q, const void *kcache, const void *vcache, const 
     if (!workspace || workspace_bytes < need) return ATFLASH_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 15u) return ATFLASH_ERR_ALIGNMENT;
     WindowParams wp;
-    if ((rc = fill_window(wp, D, rope_base, k_window, Nmax)) != ATFLASH_OK) return rc;
+    if ((rc = fill_window_theta(wp, D, theta, k_window, Nmax)) != ATFLASH_OK) return rc;
     Problem p{B, Hq, Hkv, D, Nmax};
     cudaError_t e = launch_decode(q, kcache, vcache, seqlens, out, out_dtype == ATFLASH_F32,
                                   in_dtype == ATFLASH_F32, kcache_rotated, kv_layout, p, wp,
                                   static_cast<float *>(workspace), stream);
     return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
+}
+
+int atflash_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out,
+                   int B, int Hq, int Hkv, int64_t Nmax, int D, double rope_base, double k_window,
+                   int kcache_rotated, int kv_layout, int in_dtype, int out_dtype, void *workspace,
+                   size_t workspace_bytes, cudaStream_t stream) {
+    if (!q || !kcache || !vcache || !seqlens || !out) return ATFLASH_ERR_INVALID_ARG;
+    BaseTheta bt(D, rope_base);
+    if (bt.rc != ATFLASH_OK) return bt.rc;
+    return decode_impl(q, kcache, vcache, seqlens, out, B, Hq, Hkv, Nmax, D, bt.theta, k_window, kcache_rotated,
+                       kv_layout, in_dtype, out_dtype, workspace, workspace_bytes, stream);
+}
+
+int atflash_decode_theta(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out,
+                         int B, int Hq, int Hkv, int64_t Nmax, int D, const double *theta, double k_window,
+                         int kcache_rotated, int kv_layout, int in_dtype, int out_dtype, void *workspace,
+                         size_t workspace_bytes, cudaStream_t stream) {
+    return decode_impl(q, kcache, vcache, seqlens, out, B, Hq, Hkv, Nmax, D, theta, k_window, kcache_rotated,
+                       kv_layout, in_dtype, out_dtype, workspace, workspace_bytes, stream);
 }
 
 int atflash_device_status(int clear) {

@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
     for (int r = threadIdx.x; r < H; r += kThreads) {
         sw[r] = wp.w[r];
         sTheta[r] = (float)wp.theta[r];
-        // theta_r <= 1, so the fraction is below 2^61.4 and fits the integer.
+        // theta_r <= pi (base tables: <= 1), so the fraction is at most 2^63 and fits the integer.
         sTurn[r] = __double2ull_rn(wp.theta[r] * (0.15915494309189533576888376337251 * 18446744073709551616.0));
     }
     // Rotated queries at position L-1 (fp64 angle reduction), rows >= G are zero.

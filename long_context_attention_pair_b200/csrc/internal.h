@@ -15,6 +15,9 @@ constexpr int kMaxPairs = 128;  // D <= 256
 int window_table(int D, double base, double k, int64_t N, int64_t *w);
 int pruned_terms(int64_t N, int D, double base, double k, atflash_terms *out);
 void theta_table(int D, double base, double *theta);
+bool theta_valid(int D, const double *theta);
+int window_table_theta(int D, const double *theta, double k, int64_t N, int64_t *w);
+int pruned_terms_theta(int64_t N, int D, const double *theta, double k, atflash_terms *out);
 
 // Per-call constants shared by every kernel of one call.
 struct WindowParams {

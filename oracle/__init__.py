@@ -49,8 +49,27 @@ def lib():
         L.orc_rope_rows.argtypes = [fp, i64p, i64, i, d, dp]
         L.orc_scores.argtypes = [fp, fp, i64, i, d, d, dp]
         L.orc_threads.restype = i
+        L.orc_set_theta.argtypes = [dp, i]
+        L.orc_set_theta.restype = i
         _lib = L
     return _lib
+
+
+class scaled_rope:
+    """Context manager: the oracle uses the frequency table ``theta`` (D/2 values,
+    scaled RoPE) instead of base^(-2r/D) for windows and rotations inside the block."""
+
+    def __init__(self, theta):
+        self.theta = np.ascontiguousarray(np.asarray(theta, dtype=np.float64))
+
+    def __enter__(self):
+        if lib().orc_set_theta(self.theta.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), len(self.theta)) != 0:
+            raise ValueError("oracle rejected the frequency table")
+        return self
+
+    def __exit__(self, *exc):
+        lib().orc_set_theta(None, 0)
+        return False
 
 
 def _f32(a):

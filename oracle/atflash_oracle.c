@@ -19,6 +19,12 @@
  *   s(n,m)   = (1/sqrt(D)) * sum over r with (n-m) <= w_r of t_r(n,m),  m <= n
  *   o_n      = sum_m softmax_m(s(n,.)) v_m      (two passes: max, then sums)
  *
+ * Scaled RoPE: orc_set_theta installs a caller's table theta_r (D/2 values)
+ * that replaces base^(-2r/D) in both the window (lambda_r = 2*pi/theta_r) and
+ * the rotation, until it is cleared; the definitions above are otherwise
+ * unchanged.  (The pages derive the window table from the model's RoPE
+ * configuration, "rope_scaling" included.)
+ *
  * k = +inf keeps every pair (plain causal RoPE attention).  A cell whose every
  * pair is pruned scores 0 (the empty sum), not -inf: the pages keep "the sum
  * over the rest" and drop no token.
@@ -35,12 +41,31 @@
 #endif
 
 #define ORC_TWO_PI (2.0 * 3.14159265358979323846)
+#define ORC_MAX_PAIRS 128
+
+/* Installed frequency table (scaled RoPE); orc_theta_n == 0: none. */
+static double orc_theta_tab[ORC_MAX_PAIRS];
+static int orc_theta_n = 0;
+
+/* Install theta[0..n-1] as the RoPE frequencies (n = 0 clears the table). */
+int orc_set_theta(const double *theta, int n) {
+    if (n < 0 || n > ORC_MAX_PAIRS || (n > 0 && !theta)) return -1;
+    for (int r = 0; r < n; ++r) orc_theta_tab[r] = theta[r];
+    orc_theta_n = n;
+    return 0;
+}
+
+/* theta_r: the installed table, else base^(-2r/D). */
+static double orc_theta(int r, int D, double base) {
+    if (orc_theta_n > 0 && r < orc_theta_n) return orc_theta_tab[r];
+    return pow(base, -2.0 * (double)r / (double)D);
+}
 
 /* Per-pair window limit floor(k * lambda_r) as a double (may be +inf).  The
  * pages' "w_r = k * lambda_r" with the floor of the integer-distance reading:
  * a pair is kept while the distance d satisfies d <= w_r. */
 static double orc_limit(int r, int D, double base, double kwin) {
-    double theta = pow(base, -2.0 * (double)r / (double)D);
+    double theta = orc_theta(r, D, base);
     double lambda = ORC_TWO_PI / theta;
     return floor(kwin * lambda);
 }
@@ -114,7 +139,7 @@ int64_t orc_min_kept_pairs(int64_t N, int D, double base, double kwin) {
 static void orc_rope(const float *x, int D, double base, int64_t pos, double *y) {
     int H = D / 2;
     for (int r = 0; r < H; ++r) {
-        double theta = pow(base, -2.0 * (double)r / (double)D);
+        double theta = orc_theta(r, D, base);
         double phi = (double)pos * theta;
         double c = cos(phi), s = sin(phi);
         double a = (double)x[r], b = (double)x[r + H];

@@ -216,3 +216,58 @@ def test_paged_decode_argument_errors(L):
     assert call(Hq=34, Hkv=2) == -2       # more than 16 query heads per KV head
     assert call(ws=None) == -3
     assert call(kp=ctypes.c_void_p(4100)) == -6
+
+
+# ------------------------------------------------------------------ scaled RoPE tables
+from scaled import llama3_scaled_theta  # noqa: E402
+
+
+@pytest.mark.parametrize("D,base,k,N", [(64, 1e6, 8.0, 32768), (128, 5e5, 16.0, 131072), (128, 1e7, 64.0, 1 << 20),
+                                        (64, 1e4, 1.0, 256), (128, 1e7, math.inf, 1000)])
+def test_base_table_through_theta_calls_is_bit_identical(L, D, base, k, N):
+    th = atf.theta_table(D, base)
+    assert atf.window_table(D, base, k, N) == atf.window_table(D, 0.0, k, N, theta=th)
+    assert atf.pruned_terms(N, D, base, k) == atf.pruned_terms(N, D, 0.0, k, theta=th)
+
+
+@pytest.mark.parametrize("D,base,k,N", [(128, 5e5, 16.0, 131072), (128, 5e5, 2.0, 3000), (64, 1e4, 0.5, 4096)])
+def test_scaled_window_table_equals_oracle(L, oracle, D, base, k, N):
+    th = llama3_scaled_theta(D, base)
+    with oracle.scaled_rope(th):
+        lim = oracle.window_limits(D, base, k)
+    ref = [int(min(x, N - 1)) for x in lim]
+    assert atf.window_table(D, 0.0, k, N, theta=th) == ref
+
+
+@pytest.mark.parametrize("N,D,base,k", [(700, 64, 1e4, 0.5), (300, 128, 5e5, 0.02), (2000, 128, 5e5, 1.0)])
+def test_scaled_pruned_terms_equal_bruteforce(L, oracle, N, D, base, k):
+    th = llama3_scaled_theta(D, base, factor=8.0, orig_ctx=512.0)
+    t = atf.pruned_terms(N, D, 0.0, k, theta=th)
+    with oracle.scaled_rope(th):
+        kept, total = oracle.count_bruteforce(N, D, base, k)
+    assert (t["kept"], t["total"]) == (kept, total)
+
+
+def test_theta_tables_rejected(L):
+    good = atf.theta_table(64, 1e4)
+    bad = {
+        "increasing": good[::-1],
+        "zero": [0.0] + good[1:],
+        "negative": good[:-1] + [-1e-3],
+        "nan": good[:5] + [float("nan")] + good[6:],
+        "above pi": [4.0] + good[1:],
+    }
+    for name, th in bad.items():
+        with pytest.raises(atf.AtflashError):
+            atf.window_table(64, 0.0, 1.0, 100, theta=th)
+        arr = (ctypes.c_double * 32)(*th)
+        assert L.atflash_prefill_theta(P, P, P, P, 1, 2, 1, 256, 64, arr, 1.0, atf.BF16, atf.BF16, None, P,
+                                       1 << 40, None) == -1, name
+        assert L.atflash_decode_theta(P, P, P, P, P, 1, 2, 1, 256, 64, arr, 1.0, 0, atf.KV_HND, atf.BF16,
+                                      atf.F32, P, 1 << 40, None) == -1, name
+        assert L.atflash_rope_pack_theta(P, P, 1, 256, 2, 64, arr, atf.BF16, None) == -1, name
+    assert L.atflash_prefill_theta(P, P, P, P, 1, 2, 1, 256, 64, None, 1.0, atf.BF16, atf.BF16, None, P,
+                                   1 << 40, None) == -1
+    assert L.atflash_theta_table(64, 1.0, (ctypes.c_double * 32)()) == -1
+    with pytest.raises(ValueError):
+        atf.window_table(64, 0.0, 1.0, 100, theta=good[:-1])

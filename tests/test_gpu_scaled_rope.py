@@ -1,0 +1,88 @@
+"""GPU parity of the scaled-RoPE calls (caller's frequency table instead of a base).
+
+The oracle runs with the same table installed (``oracle.scaled_rope``), which
+replaces base^(-2r/D) in its windows and rotations.  A table equal to the
+library's own base table must give bit-identical results to the base-taking
+calls.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import parity as P
+from scaled import llama3_scaled_theta
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import long_context_attention_pair_b200 as atf  # noqa: E402
+
+
+@pytest.mark.parametrize("B,N,Hq,Hkv,D,base,kwin,dtype", [
+    (1, 3000, 4, 2, 128, 5e5, 16.0, "bf16"),     # Llama-3.2-3B heads and base, scaled
+    (2, 1500, 7, 1, 64, 1e6, 2.0, "bf16"),
+    (1, 1200, 3, 3, 128, 5e5, math.inf, "bf16"),
+    (1, 300, 2, 1, 64, 1e4, 0.5, "f32"),
+])
+def test_scaled_prefill_matches_oracle(oracle, B, N, Hq, Hkv, D, base, kwin, dtype):
+    th = llama3_scaled_theta(D, base, factor=32.0, orig_ctx=min(8192.0, N / 2))
+    q = P.gen(71, "q", (B, N, Hq, D), dtype)
+    k = P.gen(71, "k", (B, N, Hkv, D), dtype)
+    v = P.gen(71, "v", (B, N, Hkv, D), dtype)
+    out = atf.prefill(q, k, v, 0.0, kwin, theta=th, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert atf.device_status() == 0
+    with oracle.scaled_rope(th):
+        ref = oracle.prefill(P.host(q), P.host(k), P.host(v), base, kwin)
+    P.check(P.host(out), ref, dtype, f"scaled prefill D={D} k={kwin}")
+
+
+@pytest.mark.parametrize("D,base,kwin", [(64, 1e6, 8.0), (128, 5e5, 16.0), (128, 1e7, math.inf)])
+def test_base_table_prefill_is_bit_identical(D, base, kwin):
+    q = P.gen(72, "q", (1, 1000, 4, D), "bf16")
+    k = P.gen(72, "k", (1, 1000, 2, D), "bf16")
+    v = P.gen(72, "v", (1, 1000, 2, D), "bf16")
+    a = atf.prefill(q, k, v, base, kwin)
+    b = atf.prefill(q, k, v, 0.0, kwin, theta=atf.theta_table(D, base))
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nmax,D,seqlens,base,kwin,layout", [
+    (2, 8, 2, 5000, 128, [5000, 1777], 5e5, 16.0, "HND"),
+    (1, 7, 1, 4097, 64, [4097], 1e6, 4.0, "NHD"),
+    (2, 28, 4, 3000, 128, [3000, 2048], 5e5, 16.0, "PACKED"),
+])
+def test_scaled_decode_matches_oracle(oracle, B, Hq, Hkv, Nmax, D, seqlens, base, kwin, layout):
+    th = llama3_scaled_theta(D, base, factor=32.0, orig_ctx=1024.0)
+    q = P.gen(73, "q_dec", (B, Hq, D), "bf16")
+    kc = P.gen(73, "k_cache", (B, Hkv, Nmax, D), "bf16")
+    vc = P.gen(73, "v_cache", (B, Hkv, Nmax, D), "bf16")
+    sl = torch.tensor(seqlens, dtype=torch.int32, device="cuda")
+    if layout == "PACKED":
+        kp = atf.rope_pack(kc.permute(0, 2, 1, 3).contiguous(), 0.0, theta=th)
+        out = atf.decode(q, kp, vc, sl, 0.0, kwin, kcache_rotated=True, kv_layout="PACKED",
+                         out_dtype=torch.float32, theta=th)
+    elif layout == "NHD":
+        out = atf.decode(q, kc.permute(0, 2, 1, 3).contiguous(), vc.permute(0, 2, 1, 3).contiguous(), sl, 0.0,
+                         kwin, kv_layout="NHD", out_dtype=torch.float32, theta=th)
+    else:
+        out = atf.decode(q, kc, vc, sl, 0.0, kwin, out_dtype=torch.float32, theta=th)
+    torch.cuda.synchronize()
+    assert atf.device_status() == 0
+    with oracle.scaled_rope(th):
+        ref = oracle.decode(P.host(q), P.host(kc), P.host(vc), seqlens, base, kwin)
+    P.check(P.host(out), ref, "bf16", f"scaled decode {layout} D={D}")
+
+
+def test_base_table_decode_is_bit_identical():
+    B, Hq, Hkv, Nmax, D, base, kwin = 2, 8, 2, 3000, 128, 1e7, 16.0
+    q = P.gen(74, "q_dec", (B, Hq, D), "bf16")
+    kc = P.gen(74, "k_cache", (B, Hkv, Nmax, D), "bf16")
+    vc = P.gen(74, "v_cache", (B, Hkv, Nmax, D), "bf16")
+    sl = torch.tensor([3000, 1234], dtype=torch.int32, device="cuda")
+    a = atf.decode(q, kc, vc, sl, base, kwin)
+    b = atf.decode(q, kc, vc, sl, 0.0, kwin, theta=atf.theta_table(D, base))
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)

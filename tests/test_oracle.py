@@ -255,3 +255,76 @@ def test_synthetic_rows_match_tensor():
     # bf16 values: low 16 bits of the float32 pattern are zero
     assert np.all((t.view(np.uint32) & 0xFFFF) == 0)
     assert abs(float(t.mean())) < 0.1 and 0.9 < float(t.std()) < 1.1
+
+
+# ------------------------------------------------------------------ scaled RoPE tables
+from scaled import base_theta, llama3_scaled_theta  # noqa: E402
+
+
+def rope_textbook_theta(x, pos, theta):
+    """Rotate-half RoPE with an explicit frequency table, matrix form."""
+    H = x.shape[-1] // 2
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * np.asarray(theta, dtype=np.float64)[None, :]
+    cos = np.concatenate([np.cos(ang), np.cos(ang)], axis=-1)
+    sin = np.concatenate([np.sin(ang), np.sin(ang)], axis=-1)
+    x = np.asarray(x, dtype=np.float64)
+    rot = np.concatenate([-x[:, H:], x[:, :H]], axis=-1)
+    return x * cos + rot * sin
+
+
+def test_scaled_table_is_a_valid_rope_table():
+    th = llama3_scaled_theta(128, 5e5)
+    assert np.all(np.diff(th) <= 0) and th[0] == 1.0 and np.all(th > 0)
+    # long wavelengths are scaled by the factor, short ones untouched
+    b = base_theta(128, 5e5)
+    assert th[-1] == b[-1] / 32.0 and th[1] == b[1]
+
+
+def test_scaled_windows_follow_the_table(oracle):
+    th = llama3_scaled_theta(128, 5e5)
+    with oracle.scaled_rope(th):
+        lim = oracle.window_limits(128, 5e5, 16.0)
+    np.testing.assert_array_equal(lim, np.floor(16.0 * 2.0 * np.pi / th))
+    # outside the block the base table is back
+    np.testing.assert_array_equal(oracle.window_limits(128, 5e5, 16.0),
+                                  np.floor(16.0 * 2.0 * np.pi / base_theta(128, 5e5)))
+
+
+@pytest.mark.parametrize("N,D,base,k", [(700, 64, 1e4, 0.5), (300, 128, 5e5, 0.02)])
+def test_scaled_count_closed_equals_bruteforce(oracle, N, D, base, k):
+    with oracle.scaled_rope(llama3_scaled_theta(D, base, factor=8.0, orig_ctx=512.0)):
+        assert oracle.count_closed(N, D, base, k) == oracle.count_bruteforce(N, D, base, k)
+
+
+def test_scaled_k_inf_is_textbook_causal_attention(oracle):
+    N, D, base = 150, 64, 1e4
+    th = llama3_scaled_theta(D, base, factor=8.0, orig_ctx=256.0)
+    q, k, v = rand((1, N, 1, D), 31), rand((1, N, 1, D), 32, "k"), rand((1, N, 1, D), 33, "v")
+    with oracle.scaled_rope(th):
+        out = oracle.prefill(q, k, v, base, math.inf)
+    pos = np.arange(N)
+    qt, kt = rope_textbook_theta(q[0, :, 0], pos, th), rope_textbook_theta(k[0, :, 0], pos, th)
+    s = qt @ kt.T / math.sqrt(D)
+    s = np.where(np.tril(np.ones((N, N), dtype=bool)), s, -np.inf)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    ref = (p / p.sum(axis=1, keepdims=True)) @ np.asarray(v[0, :, 0], dtype=np.float64)
+    np.testing.assert_allclose(out[0, :, 0], ref, rtol=0, atol=1e-12)
+
+
+def test_base_table_installed_changes_nothing(oracle):
+    N, D, base = 120, 64, 1e4
+    q, k, v = rand((1, N, 2, D), 34), rand((1, N, 1, D), 35, "k"), rand((1, N, 1, D), 36, "v")
+    plain = oracle.prefill(q, k, v, base, 1.0)
+    with oracle.scaled_rope(base_theta(D, base)):
+        tab = oracle.prefill(q, k, v, base, 1.0)
+    np.testing.assert_allclose(tab, plain, rtol=0, atol=1e-12)
+
+
+def test_scaled_decode_equals_prefill_last_row(oracle):
+    N, D, base = 200, 128, 5e5
+    th = llama3_scaled_theta(D, base, factor=8.0, orig_ctx=256.0)
+    q, k, v = rand((1, N, 4, D), 37), rand((1, N, 2, D), 38, "k"), rand((1, N, 2, D), 39, "v")
+    with oracle.scaled_rope(th):
+        pre = oracle.prefill(q, k, v, base, 0.5)
+        dec = oracle.decode(q[:, N - 1], k.transpose(0, 2, 1, 3), v.transpose(0, 2, 1, 3), [N], base, 0.5)
+    np.testing.assert_allclose(dec, pre[:, N - 1], rtol=0, atol=1e-12)

@@ -22,8 +22,8 @@ MUTANTS = {
     "rope_sign": ("y[r] = a * c - b * s;", "y[r] = a * c + b * s;"),
     "pair_index": ("qt[r + H] * kt[r + H];", "qt[r + H] * kt[r];"),
     "missing_scale": ("return acc / sqrt((double)D);", "return acc;"),
-    "theta_exponent": ("double theta = pow(base, -2.0 * (double)r / (double)D);\n    double lambda",
-                       "double theta = pow(base, -1.0 * (double)r / (double)D);\n    double lambda"),
+    "theta_exponent": ("return pow(base, -2.0 * (double)r / (double)D);",
+                       "return pow(base, -1.0 * (double)r / (double)D);"),
     "closed_form_term": ("kp += (W + 1) * (2 * (uint64_t)N - W) / 2;",
                          "kp += (W + 1) * (2 * (uint64_t)N - W + 1) / 2;"),
     "empty_sum_is_minus_inf": ("return acc / sqrt((double)D);",
