@@ -260,6 +260,15 @@ int atflash_decode_theta(const void *q, const void *kcache, const void *vcache, 
                          void *out, int B, int Hq, int Hkv, int64_t Nmax, int D, const double *theta,
                          double k_window, int kcache_rotated, int kv_layout, int in_dtype, int out_dtype,
                          void *workspace, size_t workspace_bytes, cudaStream_t stream);
+int atflash_prefill_varlen_theta(const void *q, const void *k, const void *v, void *out, const int32_t *cu_seqlens,
+                                 int B, int64_t max_seqlen, int64_t total, int Hq, int Hkv, int D,
+                                 const double *theta, double k_window, int out_dtype, float *lse, void *workspace,
+                                 size_t workspace_bytes, cudaStream_t stream);
+int atflash_decode_paged_theta(const void *q, const void *kpages, const void *vpages, const int32_t *block_table,
+                               const int32_t *seqlens, void *out, int B, int Hq, int Hkv, int max_pages,
+                               int num_pages, int page_size, int D, const double *theta, double k_window,
+                               int kcache_rotated, int kv_layout, int out_dtype, void *workspace,
+                               size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Decode that allocates nothing (no counterpart in the paper; an addition of

@@ -82,11 +82,15 @@ def lib():
         L.atflash_rope_pack_theta.argtypes = [vp, vp, i, i64, i, i, dp, i, vp]
         L.atflash_prefill_theta.argtypes = [vp, vp, vp, vp, i, i, i, i64, i, dp, d, i, i, vp, vp, sz, vp]
         L.atflash_decode_theta.argtypes = [vp, vp, vp, vp, vp, i, i, i, i64, i, dp, d, i, i, i, i, vp, sz, vp]
+        L.atflash_prefill_varlen_theta.argtypes = [vp, vp, vp, vp, vp, i, i64, i64, i, i, i, dp, d, i, vp, vp, sz, vp]
+        L.atflash_decode_paged_theta.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, dp, d, i, i, i, vp, sz,
+                                                 vp]
         for f in ("atflash_window_table", "atflash_pruned_terms", "atflash_prefill", "atflash_prefill_ex",
                   "atflash_decode", "atflash_device_status", "atflash_rope_pack", "atflash_prefill_packed",
                   "atflash_prefill_varlen", "atflash_decode_paged", "atflash_theta_table",
                   "atflash_window_table_theta", "atflash_pruned_terms_theta", "atflash_rope_pack_theta",
-                  "atflash_prefill_theta", "atflash_decode_theta"):
+                  "atflash_prefill_theta", "atflash_decode_theta", "atflash_prefill_varlen_theta",
+                  "atflash_decode_paged_theta"):
             getattr(L, f).restype = i
         _lib = L
     return _lib
@@ -210,7 +214,7 @@ def prefill(q, k, v, rope_base: float, k_window: float = math.inf, *, out=None, 
 
 
 def prefill_varlen(q, k, v, cu_seqlens, max_seqlen: int, rope_base: float, k_window: float = math.inf, *,
-                   out=None, out_dtype=None, return_lse: bool = False, workspace=None, stream=None):
+                   out=None, out_dtype=None, return_lse: bool = False, workspace=None, stream=None, theta=None):
     """Windowed causal RoPE prefill of a ragged batch packed along the token axis.
 
     q [total, Hq, D], k/v [total, Hkv, D] bf16 (un-rotated); cu_seqlens int32 [B+1]
@@ -231,18 +235,21 @@ def prefill_varlen(q, k, v, cu_seqlens, max_seqlen: int, rope_base: float, k_win
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
-    st = lib().atflash_prefill_varlen(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
-                                      _dev(cu_seqlens, "cu_seqlens"), B, int(max_seqlen), total, Hq, Hkv, D,
-                                      float(rope_base), float(k_window), _dtype_code(out),
-                                      _dev(lse, "lse") if lse is not None else None, ws_ptr,
-                                      ws_bytes if workspace is not None else need, _stream_ptr(stream))
-    _check(st, "atflash_prefill_varlen")
+    fn, name = lib().atflash_prefill_varlen, "atflash_prefill_varlen"
+    rope = float(rope_base)
+    if theta is not None:
+        fn, name, rope = lib().atflash_prefill_varlen_theta, "atflash_prefill_varlen_theta", _theta_arg(theta, D)
+    st = fn(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(cu_seqlens, "cu_seqlens"), B,
+            int(max_seqlen), total, Hq, Hkv, D, rope, float(k_window), _dtype_code(out),
+            _dev(lse, "lse") if lse is not None else None, ws_ptr, ws_bytes if workspace is not None else need,
+            _stream_ptr(stream))
+    _check(st, name)
     return (out, lse) if return_lse else out
 
 
 def decode_paged(q, kpages, vpages, block_table, seqlens, page_size: int, rope_base: float,
                  k_window: float = math.inf, *, kcache_rotated: bool = False, kv_layout: str = "NHD", out=None,
-                 out_dtype=None, workspace=None, stream=None):
+                 out_dtype=None, workspace=None, stream=None, theta=None):
     """One decode step over a paged KV cache.
 
     q [B, Hq, D] bf16; block_table int32 [B, max_pages]; seqlens int32 [B].
@@ -261,12 +268,15 @@ def decode_paged(q, kpages, vpages, block_table, seqlens, page_size: int, rope_b
     need = decode_workspace_bytes(B, Hq, Hkv, max_pages * page_size, D)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    st = lib().atflash_decode_paged(_dev(q, "q"), _dev(kpages, "kpages"), _dev(vpages, "vpages"),
-                                    _dev(block_table, "block_table"), _dev(seqlens, "seqlens"), _dev(out, "out"), B,
-                                    Hq, Hkv, max_pages, num_pages, int(page_size), D, float(rope_base),
-                                    float(k_window), 1 if kcache_rotated else 0, lay, _dtype_code(out),
-                                    _dev(workspace, "workspace"), need, _stream_ptr(stream))
-    _check(st, "atflash_decode_paged")
+    fn, name = lib().atflash_decode_paged, "atflash_decode_paged"
+    rope = float(rope_base)
+    if theta is not None:
+        fn, name, rope = lib().atflash_decode_paged_theta, "atflash_decode_paged_theta", _theta_arg(theta, D)
+    st = fn(_dev(q, "q"), _dev(kpages, "kpages"), _dev(vpages, "vpages"), _dev(block_table, "block_table"),
+            _dev(seqlens, "seqlens"), _dev(out, "out"), B, Hq, Hkv, max_pages, num_pages, int(page_size), D, rope,
+            float(k_window), 1 if kcache_rotated else 0, lay, _dtype_code(out), _dev(workspace, "workspace"), need,
+            _stream_ptr(stream))
+    _check(st, name)
     return out
 
 

@@ -119,14 +119,6 @@ static int fill_window_theta(WindowParams &wp, int D, const double *theta, doubl
     return ATFLASH_OK;
 }
 
-static int fill_window(WindowParams &wp, int D, double base, double k, int64_t N) {
-    int rc = check_window_args(D, base, k);
-    if (rc != ATFLASH_OK) return rc;
-    double theta[kMaxPairs];
-    theta_table(D, base, theta);
-    return fill_window_theta(wp, D, theta, k, N);
-}
-
 static size_t prefill_ws(int B, int Hq, int Hkv, int64_t N, int D, int in_dtype) {
     const size_t es = (in_dtype == ATFLASH_F32) ? 4 : 2;
     return align256((size_t)B * Hq * N * D * es) + align256((size_t)B * Hkv * N * D * es);
@@ -337,12 +329,12 @@ int atflash_prefill(const void *q, const void *k, const void *v, void *out, int 
     return rc;
 }
 
-static int check_varlen(int B, int Hq, int Hkv, int64_t max_seqlen, int64_t total, int D, double base, double k,
-                        int out_dtype) {
+static int check_varlen(int B, int Hq, int Hkv, int64_t max_seqlen, int64_t total, int D, const double *theta,
+                        double k, int out_dtype) {
     int rc = check_shape(B, Hq, Hkv, max_seqlen);
     if (rc != ATFLASH_OK) return rc;
     if (total < 1 || total > INT32_MAX || max_seqlen > total) return ATFLASH_ERR_INVALID_ARG;
-    if ((rc = check_window_args(D, base, k)) != ATFLASH_OK) return rc;
+    if ((rc = check_theta_args(D, theta, k)) != ATFLASH_OK) return rc;
     if (D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
     if (out_dtype != ATFLASH_F32 && out_dtype != ATFLASH_BF16) return ATFLASH_ERR_UNSUPPORTED;
     return ATFLASH_OK;
@@ -353,12 +345,12 @@ size_t atflash_prefill_varlen_workspace_bytes(int Hq, int Hkv, int64_t total, in
     return align256((size_t)Hq * total * D * 2) + align256((size_t)Hkv * total * D * 2);
 }
 
-int atflash_prefill_varlen(const void *q, const void *k, const void *v, void *out, const int32_t *cu_seqlens, int B,
-                           int64_t max_seqlen, int64_t total, int Hq, int Hkv, int D, double rope_base,
-                           double k_window, int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
-                           cudaStream_t stream) {
+static int prefill_varlen_impl(const void *q, const void *k, const void *v, void *out, const int32_t *cu_seqlens,
+                               int B, int64_t max_seqlen, int64_t total, int Hq, int Hkv, int D, const double *theta,
+                               double k_window, int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
     if (!q || !k || !v || !out || !cu_seqlens) return ATFLASH_ERR_INVALID_ARG;
-    int rc = check_varlen(B, Hq, Hkv, max_seqlen, total, D, rope_base, k_window, out_dtype);
+    int rc = check_varlen(B, Hq, Hkv, max_seqlen, total, D, theta, k_window, out_dtype);
     if (rc != ATFLASH_OK) return rc;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATFLASH_ERR_ALIGNMENT;
     const size_t need = atflash_prefill_varlen_workspace_bytes(Hq, Hkv, total, D);
@@ -377,7 +369,7 @@ int atflash_prefill_varlen(const void *q, const void *k, const void *v, void *ou
     void *qt = ws;
     void *kt = ws + align256((size_t)Hq * total * D * 2);
     WindowParams wp;
-    rc = fill_window(wp, D, rope_base, k_window, max_seqlen);
+    rc = fill_window_theta(wp, D, theta, k_window, max_seqlen);
     cudaError_t e = cudaSuccess;
     int *status = device_status_word();
     if (rc == ATFLASH_OK && !status) rc = ATFLASH_ERR_CUDA;
@@ -394,22 +386,42 @@ int atflash_prefill_varlen(const void *q, const void *k, const void *v, void *ou
     return rc;
 }
 
+int atflash_prefill_varlen(const void *q, const void *k, const void *v, void *out, const int32_t *cu_seqlens, int B,
+                           int64_t max_seqlen, int64_t total, int Hq, int Hkv, int D, double rope_base,
+                           double k_window, int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+    if (!q || !k || !v || !out || !cu_seqlens) return ATFLASH_ERR_INVALID_ARG;
+    BaseTheta bt(D, rope_base);
+    if (bt.rc != ATFLASH_OK) return bt.rc;
+    return prefill_varlen_impl(q, k, v, out, cu_seqlens, B, max_seqlen, total, Hq, Hkv, D, bt.theta, k_window,
+                               out_dtype, lse, workspace, workspace_bytes, stream);
+}
+
+int atflash_prefill_varlen_theta(const void *q, const void *k, const void *v, void *out, const int32_t *cu_seqlens,
+                                 int B, int64_t max_seqlen, int64_t total, int Hq, int Hkv, int D,
+                                 const double *theta, double k_window, int out_dtype, float *lse, void *workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+    return prefill_varlen_impl(q, k, v, out, cu_seqlens, B, max_seqlen, total, Hq, Hkv, D, theta, k_window,
+                               out_dtype, lse, workspace, workspace_bytes, stream);
+}
+
 size_t atflash_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D) {
     if (check_shape(B, Hq, Hkv, Nmax) != ATFLASH_OK || (D != 64 && D != 128)) return 0;
     return decode_workspace_bytes(B, Hq, Hkv, Nmax, D);
 }
 
-int atflash_decode_paged(const void *q, const void *kpages, const void *vpages, const int32_t *block_table,
-                         const int32_t *seqlens, void *out, int B, int Hq, int Hkv, int max_pages, int num_pages,
-                         int page_size, int D, double rope_base, double k_window, int kcache_rotated, int kv_layout,
-                         int out_dtype, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+static int decode_paged_impl(const void *q, const void *kpages, const void *vpages, const int32_t *block_table,
+                             const int32_t *seqlens, void *out, int B, int Hq, int Hkv, int max_pages, int num_pages,
+                             int page_size, int D, const double *theta, double k_window, int kcache_rotated,
+                             int kv_layout, int out_dtype, void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream) {
     if (!q || !kpages || !vpages || !block_table || !seqlens || !out) return ATFLASH_ERR_INVALID_ARG;
     if (max_pages < 1 || num_pages < 1 || page_size < 64 || page_size % 64 != 0) return ATFLASH_ERR_INVALID_ARG;
     const int64_t Nmax = (int64_t)max_pages * page_size;
     int rc = check_shape(B, Hq, Hkv, Nmax);
     if (rc != ATFLASH_OK) return rc;
     if ((int64_t)num_pages * Hkv * (D / 16) > INT32_MAX) return ATFLASH_ERR_INVALID_ARG;
-    if ((rc = check_window_args(D, rope_base, k_window)) != ATFLASH_OK) return rc;
+    if ((rc = check_theta_args(D, theta, k_window)) != ATFLASH_OK) return rc;
     if (kcache_rotated != 0 && kcache_rotated != 1) return ATFLASH_ERR_INVALID_ARG;
     if (kv_layout != ATFLASH_KV_NHD && kv_layout != ATFLASH_KV_PACKED) return ATFLASH_ERR_INVALID_ARG;
     if (kv_layout == ATFLASH_KV_PACKED && !kcache_rotated) return ATFLASH_ERR_INVALID_ARG;
@@ -421,12 +433,34 @@ int atflash_decode_paged(const void *q, const void *kpages, const void *vpages, 
     if (!workspace || workspace_bytes < need) return ATFLASH_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 15u) return ATFLASH_ERR_ALIGNMENT;
     WindowParams wp;
-    if ((rc = fill_window(wp, D, rope_base, k_window, Nmax)) != ATFLASH_OK) return rc;
+    if ((rc = fill_window_theta(wp, D, theta, k_window, Nmax)) != ATFLASH_OK) return rc;
     Problem p{B, Hq, Hkv, D, Nmax};
     PagedKV pk{block_table, max_pages, page_size, num_pages};
     cudaError_t e = launch_decode(q, kpages, vpages, seqlens, out, out_dtype == ATFLASH_F32, 0, kcache_rotated,
                                   kv_layout, p, wp, static_cast<float *>(workspace), stream, &pk);
     return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
+}
+
+int atflash_decode_paged(const void *q, const void *kpages, const void *vpages, const int32_t *block_table,
+                         const int32_t *seqlens, void *out, int B, int Hq, int Hkv, int max_pages, int num_pages,
+                         int page_size, int D, double rope_base, double k_window, int kcache_rotated, int kv_layout,
+                         int out_dtype, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (!q || !kpages || !vpages || !block_table || !seqlens || !out) return ATFLASH_ERR_INVALID_ARG;
+    BaseTheta bt(D, rope_base);
+    if (bt.rc != ATFLASH_OK) return bt.rc;
+    return decode_paged_impl(q, kpages, vpages, block_table, seqlens, out, B, Hq, Hkv, max_pages, num_pages,
+                             page_size, D, bt.theta, k_window, kcache_rotated, kv_layout, out_dtype, workspace,
+                             workspace_bytes, stream);
+}
+
+int atflash_decode_paged_theta(const void *q, const void *kpages, const void *vpages, const int32_t *block_table,
+                               const int32_t *seqlens, void *out, int B, int Hq, int Hkv, int max_pages,
+                               int num_pages, int page_size, int D, const double *theta, double k_window,
+                               int kcache_rotated, int kv_layout, int out_dtype, void *workspace,
+                               size_t workspace_bytes, cudaStream_t stream) {
+    return decode_paged_impl(q, kpages, vpages, block_table, seqlens, out, B, Hq, Hkv, max_pages, num_pages,
+                             page_size, D, theta, k_window, kcache_rotated, kv_layout, out_dtype, workspace,
+                             workspace_bytes, stream);
 }
 
 static int decode_impl(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out,

@@ -86,3 +86,38 @@ def test_base_table_decode_is_bit_identical():
     b = atf.decode(q, kc, vc, sl, 0.0, kwin, theta=atf.theta_table(D, base))
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_scaled_varlen_prefill_matches_oracle(oracle):
+    import test_gpu_varlen as VL
+    lens, Hq, Hkv, D, base, kwin = [700, 1, 1300], 4, 2, 128, 5e5, 2.0
+    th = llama3_scaled_theta(D, base, factor=32.0, orig_ctx=512.0)
+    q, k, v, cu = VL.packed_batch(75, lens, Hq, Hkv, D)
+    cu_d = torch.as_tensor(cu, device="cuda")
+    out = atf.prefill_varlen(q, k, v, cu_d, max(lens), 0.0, kwin, out_dtype=torch.float32, theta=th)
+    base_out = atf.prefill_varlen(q, k, v, cu_d, max(lens), base, kwin, out_dtype=torch.float32)
+    same = atf.prefill_varlen(q, k, v, cu_d, max(lens), 0.0, kwin, out_dtype=torch.float32,
+                              theta=atf.theta_table(D, base))
+    torch.cuda.synchronize()
+    assert atf.device_status() == 0
+    assert torch.equal(same, base_out)
+    with oracle.scaled_rope(th):
+        VL.check_against_oracle(oracle, q, k, v, cu, out, base, kwin)
+
+
+def test_scaled_paged_decode_equals_contiguous_scaled_decode():
+    import test_gpu_paged as PG
+    B, Hq, Hkv, L, D, P_, base, kwin = 2, 8, 2, 2048, 128, 64, 5e5, 4.0
+    th = llama3_scaled_theta(D, base, factor=32.0, orig_ctx=1024.0)
+    q = P.gen(76, "q_dec", (B, Hq, D), "bf16")
+    kc = P.gen(76, "k_cache", (B, Hkv, L, D), "bf16")
+    vc = P.gen(76, "v_cache", (B, Hkv, L, D), "bf16")
+    sl = torch.tensor([2048, 999], dtype=torch.int32, device="cuda")
+    ids, n_pool = PG.scatter_pages(B, Hkv, L, P_, 77)
+    bt = torch.as_tensor(ids, device="cuda")
+    kpool, vpool = PG.nhd_pool(kc, ids, n_pool, P_), PG.nhd_pool(vc, ids, n_pool, P_)
+    ref = atf.decode(q, kc, vc, sl, 0.0, kwin, out_dtype=torch.float32, theta=th)
+    out = atf.decode_paged(q, kpool, vpool, bt, sl, P_, 0.0, kwin, out_dtype=torch.float32, theta=th)
+    torch.cuda.synchronize()
+    assert atf.device_status() == 0
+    assert torch.equal(out, ref)
