@@ -88,8 +88,8 @@ TRAFFIC = {"bytes_per_launch": 99188992, "source_sha1": "67d3d80e1932ab93afb73bd
 # the full-size workload, from one single-pass ncu capture
 # (profiles/decode_tc_qwen7b_packed_4x128k.md); valid while decode_tc.cu hashes to
 # `source_sha1`.
-DECODE_TRAFFIC = {"decode_1m_packed": {"bytes_per_launch": 6607551744,
-                                       "source_sha1": "60819fd860ef68921aa18d358fbc1c8b40b9508a"}}
+DECODE_TRAFFIC = {"decode_1m_packed": {"bytes_per_launch": 6607405312,
+                                       "source_sha1": "ad7ae6e989545528735e37df19aea04010f4cad1"}}
 
 
 def parse():

@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
     __shared__ int sw[kMaxPairs];
     __shared__ float sTheta[kMaxPairs];
     __shared__ uint64_t sTurn[kMaxPairs];  // theta_r / (2*pi) in units of 2^-64 turns
+    __shared__ float2 sRot8[kMaxPairs];    // (cos, sin) of 8 * theta_r (rotation at load)
 
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_);
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -173,6 +174,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
         sTheta[r] = (float)wp.theta[r];
         // theta_r <= pi (base tables: <= 1), so the fraction is at most 2^63 and fits the integer.
         sTurn[r] = __double2ull_rn(wp.theta[r] * (0.15915494309189533576888376337251 * 18446744073709551616.0));
+        if (!kPacked && !krot) {
+            double s8, c8;
+            sincos(8.0 * wp.theta[r], &s8, &c8);
+            sRot8[r] = make_float2((float)c8, (float)s8);
+        }
     }
     // Rotated queries at position L-1 (fp64 angle reduction), rows >= G are zero.
     for (int e = threadIdx.x; e < 16 * H; e += kThreads) {
@@ -355,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
                 const int c_warp = r_warp >> 3;
                 // Distances of this thread's keys kw0 + gq and kw0 + gq + 8.
                 const int da = Lq - (kw0 + gq), db = da - 8;
-                const float fa = (float)(16 * wq + gq), fb = fa + 8.f;
+                const float fa = (float)(16 * wq + gq);
                 const uint32_t kst = sKa + st * F::KBytes;
                 const int mi = lane >> 3, ri = lane & 7;
                 const int c_keep = (r_keep + 7) >> 3;
@@ -425,15 +431,22 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
                         } else {
                             const float th0 = sTheta[p0], th1 = sTheta[p1];
                             const float base0 = sBase[st * H + p0], base1 = sBase[st * H + p1];
-                            float ang[4] = {fmaf(fa, th0, base0), fmaf(fa, th1, base1), fmaf(fb, th0, base0),
-                                            fmaf(fb, th1, base1)};
+                            // Key gq's angles reduced to [-pi, pi] and sin/cos taken; key gq+8
+                            // sits 8 positions later: its (cos, sin) is key gq's rotated by the
+                            // fixed 8*theta_r (angle addition, 4 FMAs instead of a sincos).
+                            float ang[2] = {fmaf(fa, th0, base0), fmaf(fa, th1, base1)};
                             float cs[4], sn[4];
 #pragma unroll
-                            for (int u = 0; u < 4; ++u) {
+                            for (int u = 0; u < 2; ++u) {
                                 const float turns = rintf(ang[u] * 0.15915494309189533577f);
                                 const float x = fmaf(-turns, 6.283185307179586477f, ang[u]);
                                 __sincosf(x, &sn[u], &cs[u]);
                             }
+                            const float2 e0 = sRot8[p0], e1 = sRot8[p1];
+                            cs[2] = fmaf(cs[0], e0.x, -sn[0] * e0.y);
+                            sn[2] = fmaf(sn[0], e0.x, cs[0] * e0.y);
+                            cs[3] = fmaf(cs[1], e1.x, -sn[1] * e1.y);
+                            sn[3] = fmaf(sn[1], e1.x, cs[1] * e1.y);
                             rotate_pairs(b0, b1, cs[0], sn[0], cs[1], sn[1], ka0, ka1);
                             rotate_pairs(b2, b3, cs[2], sn[2], cs[3], sn[3], kb0, kb1);
                         }
