@@ -89,7 +89,7 @@ TRAFFIC = {"bytes_per_launch": 99188992, "source_sha1": "67d3d80e1932ab93afb73bd
 # (profiles/decode_tc_qwen7b_packed_4x128k.md); valid while decode_tc.cu hashes to
 # `source_sha1`.
 DECODE_TRAFFIC = {"decode_1m_packed": {"bytes_per_launch": 6607405312,
-                                       "source_sha1": "ad7ae6e989545528735e37df19aea04010f4cad1"}}
+                                       "source_sha1": "d7b5169d59996c1a554d660578c2ccb20b0d7d15"}}
 
 
 def parse():

@@ -1,7 +1,8 @@
 // Split-KV windowed decode on tensor cores (bf16 caches).
 //
-// One CTA = one split of one (sequence, KV head): its G = Hq/Hkv query heads
-// are the M rows (padded to 16) of mma.sync m16n8k16 tiles, keys are N.  The
+// One CTA = one split of one (sequence, KV head): the 16 keys of a consumer
+// warp are the M rows of mma.sync m16n8k16 tiles and the G = Hq/Hkv query
+// heads their N columns (tiles of 8 heads).  The
 // method ("ATFlash — Per-RoPE-Wavelength Attention Windows", "The idea" and
 // "Numbers": the window is a condition on which K elements are loaded):
 // for a key at distance d = L-1-m only pairs r >= r*(d) are kept, so
@@ -10,7 +11,7 @@
 //   - each consumer warp takes 16 keys of a stage: ldmatrix puts complete
 //     frequency pairs (r, r+D/2) of one key into one thread, which rotates them
 //     (unless the cache is pre-rotated) and zeroes the pairs its key prunes;
-//   - S = Q~ K~^T, the online softmax and O += P V stay in registers.
+//   - S^T = K~ Q~^T, the online softmax and O^T += V^T P^T stay in registers.
 // The contraction order inside a K-step is [8 low-half dims, 8 high-half dims]
 // for both Q~ and K~, so every dot product is unchanged.
 //
