@@ -55,6 +55,8 @@ SMALL = [
     # groups of 9..16 heads take two 8-head tiles of the MMA's N
     (2, 24, 2, 2100, 128, [2100, 1500], 5e5, 16.0, 0, "bf16"),
     (1, 10, 1, 1300, 64, [1300], 1e4, 2.0, 1, "bf16"),
+    # k = 0: only the query's own position keeps its pairs
+    (2, 8, 2, 900, 128, [900, 333], 1e4, 0.0, 0, "bf16"),
 ]
 
 
@@ -80,6 +82,7 @@ def test_decode_matches_oracle(oracle, B, Hq, Hkv, Nmax, D, seqlens, base, kwin,
     # two head tiles at D = 128; a cache length that is not a multiple of 4
     (2, 24, 2, 2102, 128, [2102, 999], 5e5, 16.0),
     (1, 12, 1, 2048, 128, [2048], 1e4, 4.0),
+    (2, 8, 2, 1000, 64, [1000, 65], 1e4, 0.0),
 ])
 def test_packed_rotated_cache_matches_oracle(oracle, B, Hq, Hkv, Nmax, D, seqlens, base, kwin):
     # The RoPE pre-pass writes the packed cache from the un-rotated keys; the oracle

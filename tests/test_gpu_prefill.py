@@ -54,6 +54,11 @@ SMALL_BF16 = [
     (1, 1000, 128, 2, 1, 1e4, math.inf),
     (1, 513, 64, 7, 1, 1e6, math.inf),
     (1, 2048, 128, 2, 1, 1e4, 0.5),
+    # k = 0: only distance 0 keeps its pairs, every other cell is the empty sum 0
+    (1, 600, 64, 2, 1, 1e4, 0.0),
+    (1, 400, 128, 4, 2, 5e5, 0.0),
+    # window off at D = 64 with an even GQA group (one head per CTA, two CTAs per SM)
+    (2, 640, 64, 4, 2, 1e4, math.inf),
 ]
 
 
