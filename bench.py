@@ -54,7 +54,41 @@ WORKLOADS = {
                        1, 28, 4, 128, 524288, 1e7, 16.0, 3),
     "qwen7b_512k_k64": _pf("Qwen2.5-7B-1M-shaped single-layer windowed prefill + decode of the last row",
                            1, 28, 4, 128, 524288, 1e7, 64.0, 3),
+    # Llama-3.2-3B as released: its RoPE frequencies rescaled (rope_scaling type llama3,
+    # factor 32, low/high frequency factors 1 and 4, original context 8192).  Only pairs
+    # with wavelengths above 2048 are rescaled, and at k = 16 their windows exceed
+    # 32K already, so the scaled table changes the windows only beyond 32K tokens.
+    "llama3b_128k_scaled": dict(_pf("Llama-3.2-3B-shaped single-layer windowed prefill + decode of the last row, "
+                                    "llama3 rope_scaling", 1, 24, 8, 128, 131072, 5e5, 16.0, 2),
+                                rope_scaling={"factor": 32.0, "low_freq_factor": 1.0, "high_freq_factor": 4.0,
+                                              "original_max_position_embeddings": 8192}),
 }
+
+
+def rope_theta(wl):
+    """Per-pair frequencies of a workload with rope_scaling (None: base^(-2r/D)).
+
+    The llama3 rule: a pair whose wavelength 2*pi/theta_r is shorter than
+    orig/high keeps its frequency, one longer than orig/low has it divided by
+    `factor`, and in between the two are blended linearly in orig/wavelength."""
+    sc = wl.get("rope_scaling")
+    if not sc:
+        return None
+    D, base = wl["D"], wl["rope_base"]
+    f, lo, hi = sc["factor"], sc["low_freq_factor"], sc["high_freq_factor"]
+    orig = float(sc["original_max_position_embeddings"])
+    out = []
+    for r in range(D // 2):
+        th = base ** (-2.0 * r / D)
+        wavelen = 2.0 * math.pi / th
+        if wavelen < orig / hi:
+            out.append(th)
+        elif wavelen > orig / lo:
+            out.append(th / f)
+        else:
+            a = (orig / wavelen - lo) / (hi - lo)
+            out.append((1.0 - a) * th / f + a * th)
+    return out
 # Decode workloads: one step = one decode call (one token for each of B sequences).
 DECODE_WORKLOADS = {
     "decode_1m": {"workload": "Qwen2.5-7B-1M-shaped decode, 4 sequences at 1M tokens", "B": 4, "Hq": 28,
@@ -75,6 +109,27 @@ DECODE_WORKLOADS = {
     "decode_128k_k64": {"workload": "Qwen2.5-7B-1M-shaped decode, 16 sequences at 128K tokens", "B": 16,
                         "Hq": 28, "Hkv": 4, "D": 128, "N": 1 << 17, "rope_base": 1e7, "k_window": 64.0,
                         "seed": 5},
+    # Paged caches: the contiguous cache cut into pages of `page` tokens and scattered
+    # through one pool in a seeded random order (block table per sequence).
+    "decode_1m_paged_packed": {"workload": "Qwen2.5-7B-1M-shaped decode, 4 sequences at 1M tokens, paged packed "
+                               "rotated K cache (256-token pages, shuffled pool)", "B": 4, "Hq": 28, "Hkv": 4,
+                               "D": 128, "N": 1 << 20, "rope_base": 1e7, "k_window": 16.0, "seed": 4,
+                               "packed": True, "page": 256},
+    "decode_1m_paged": {"workload": "Qwen2.5-7B-1M-shaped decode, 4 sequences at 1M tokens, paged NHD cache "
+                        "(256-token pages, shuffled pool)", "B": 4, "Hq": 28, "Hkv": 4, "D": 128, "N": 1 << 20,
+                        "rope_base": 1e7, "k_window": 16.0, "seed": 4, "page": 256},
+}
+# Ragged-batch prefill workloads: one step = one varlen prefill call (RoPE pre-pass of
+# the packed Q and K, then the windowed prefill) over sequences of mixed lengths.
+VARLEN_WORKLOADS = {
+    "varlen_qwen05b_256k": {"workload": "Qwen2.5-0.5B-shaped single-layer windowed prefill of a ragged batch, "
+                            "lengths log-uniform in [1K, 64K] tokens, 256K tokens in all", "Hq": 14, "Hkv": 2,
+                            "D": 64, "total": 1 << 18, "len_lo": 1024, "len_hi": 65536, "rope_base": 1e6,
+                            "k_window": 8.0, "seed": 6},
+    "varlen_qwen7b_1m": {"workload": "Qwen2.5-7B-1M-shaped single-layer windowed prefill of a ragged batch, "
+                         "lengths log-uniform in [4K, 256K] tokens, 1M tokens in all", "Hq": 28, "Hkv": 4,
+                         "D": 128, "total": 1 << 20, "len_lo": 4096, "len_hi": 262144, "rope_base": 1e7,
+                         "k_window": 16.0, "seed": 7},
 }
 WORKLOAD = WORKLOADS["qwen05b_32k"]
 L2_FLUSH_BYTES = 256 << 20
@@ -83,13 +138,16 @@ KERNELS_PER_STEP = 5  # rope_pack(q), rope_pack(k), prefill_tc, decode_split, de
 # DRAM bytes per launch of the tcgen05 prefill kernel on this workload, from one
 # ncu capture (profiles/prefill_tc_qwen05b_32k.md).  Valid only while the
 # kernel source hashes to `source_sha1`; otherwise the line reports null.
-TRAFFIC = {"bytes_per_launch": 99188992, "source_sha1": "67d3d80e1932ab93afb73bd40c88732f7a2d323c"}
+TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 99188992,
+           "source_sha1": "67d3d80e1932ab93afb73bd40c88732f7a2d323c"}
 # DRAM bytes per launch of the decode kernel (split states included, merge not) on
-# the full-size workload, from one single-pass ncu capture
+# the full-size workloads, from single-pass ncu captures
 # (profiles/decode_tc_qwen7b_packed_4x128k.md); valid while decode_tc.cu hashes to
 # `source_sha1`.
 DECODE_TRAFFIC = {"decode_1m_packed": {"bytes_per_launch": 6607405312,
-                                       "source_sha1": "d7b5169d59996c1a554d660578c2ccb20b0d7d15"}}
+                                       "source_sha1": "d7b5169d59996c1a554d660578c2ccb20b0d7d15"},
+                  "decode_1m": {"bytes_per_launch": 8608839424,
+                                "source_sha1": "d7b5169d59996c1a554d660578c2ccb20b0d7d15"}}
 
 
 def parse():
@@ -101,7 +159,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--workload", default="qwen05b_32k",
-                   choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS))
+                   choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(VARLEN_WORKLOADS))
     p.add_argument("--N", type=int, default=None, help="override sequence length (sweeps)")
     p.add_argument("--k-window", type=float, default=None, help="override k (inf = window off)")
     return p.parse_args()
@@ -123,6 +181,17 @@ def kernel_sha1(name="prefill_tc.cu"):
 
 
 # ---------------------------------------------------------------- distributed
+def prefill_traffic(workload, wl):
+    """Captured DRAM bytes of one prefill launch, for the workload (at its own N
+    and k) and kernel source the capture was made on; otherwise None."""
+    if workload != TRAFFIC["workload"] or TRAFFIC["source_sha1"] != kernel_sha1():
+        return None
+    ref = WORKLOADS[workload]
+    if wl["N"] != ref["N"] or wl["k_window"] != ref["k_window"]:
+        return None
+    return TRAFFIC["bytes_per_launch"]
+
+
 def decode_traffic(workload, L):
     """Captured DRAM bytes of one decode launch for this workload, or None."""
     rec = DECODE_TRAFFIC.get(workload)
@@ -230,8 +299,10 @@ class ClockSampler:
 # ----------------------------------------------------------------- CPU oracle
 def cpu_baseline(q, k, v, wl, budget_s=12.0):
     """The fp64 oracle, as it stands, on a bounded sample of query rows (all heads)."""
+    import contextlib
     import numpy as np
     import oracle
+    th = rope_theta(wl)
     N = wl["N"]
     kh = k[0].float().cpu().numpy()
     vh = v[0].float().cpu().numpy()
@@ -241,7 +312,8 @@ def cpu_baseline(q, k, v, wl, budget_s=12.0):
         rows = np.sort(rng.choice(N, size=nrows, replace=False))
         qh = q[0, rows].float().cpu().numpy()
         t0 = time.perf_counter()
-        oracle.prefill_rows(qh, rows, kh, vh, wl["rope_base"], wl["k_window"])
+        with (oracle.scaled_rope(th) if th is not None else contextlib.nullcontext()):
+            oracle.prefill_rows(qh, rows, kh, vh, wl["rope_base"], wl["k_window"])
         return time.perf_counter() - t0
 
     t = run(8)
@@ -267,10 +339,16 @@ def run_reference(args, wl):
     rng = np.random.default_rng(99)
     qshape = (wl["B"], N, wl["Hq"], wl["D"])
 
+    th = rope_theta(wl)
+
     def step():
         rows = np.sort(rng.choice(N, size=rows_per_step, replace=False))
         qr = synthetic.rows(wl["seed"], "q", qshape, 1, rows, "bf16")[0]
-        oracle.prefill_rows(qr, rows, k, v, wl["rope_base"], wl["k_window"])
+        if th is None:
+            oracle.prefill_rows(qr, rows, k, v, wl["rope_base"], wl["k_window"])
+        else:
+            with oracle.scaled_rope(th):
+                oracle.prefill_rows(qr, rows, k, v, wl["rope_base"], wl["k_window"])
 
     for _ in range(args.warmup):
         step()
@@ -304,6 +382,8 @@ def run_ours(args, wl):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     B, N, Hq, Hkv, D = wl["B"], wl["N"], wl["Hq"], wl["Hkv"], wl["D"]
     base, kwin = wl["rope_base"], wl["k_window"]
+    th = rope_theta(wl)
+    tk = {} if th is None else {"theta": th}
     q = synthetic.tensor_torch(wl["seed"], "q", (B, N, Hq, D), "bf16", device=dev)
     k = synthetic.tensor_torch(wl["seed"], "k", (B, N, Hkv, D), "bf16", device=dev)
     v = synthetic.tensor_torch(wl["seed"], "v", (B, N, Hkv, D), "bf16", device=dev)
@@ -318,14 +398,14 @@ def run_ours(args, wl):
     stream = torch.cuda.current_stream()
 
     def step(kw, ev=None):
-        atf.rope_pack(q, base, out=qpack)
-        atf.rope_pack(k, base, out=kpack)
+        atf.rope_pack(q, base, out=qpack, **tk)
+        atf.rope_pack(k, base, out=kpack, **tk)
         if ev is not None:
             ev[0].record(stream)
-        atf.prefill_packed(qpack, kpack, v, base, kw, out=out)
+        atf.prefill_packed(qpack, kpack, v, base, kw, out=out, **tk)
         if ev is not None:
             ev[1].record(stream)
-        atf.decode(q_last, k, v, seqlens, base, kw, kv_layout="NHD", out=dec_out, workspace=dws)
+        atf.decode(q_last, k, v, seqlens, base, kw, kv_layout="NHD", out=dec_out, workspace=dws, **tk)
 
     def timed(kw, steps):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -366,7 +446,7 @@ def run_ours(args, wl):
     for a, b in dec_ev:
         flush.zero_()
         a.record(stream)
-        atf.decode(q_last, k, v, seqlens, base, kwin, kv_layout="NHD", out=dec_out, workspace=dws)
+        atf.decode(q_last, k, v, seqlens, base, kwin, kv_layout="NHD", out=dec_out, workspace=dws, **tk)
         b.record(stream)
     torch.cuda.synchronize()
     dec_us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in dec_ev)
@@ -377,13 +457,13 @@ def run_ours(args, wl):
     off_ms_per_step = off_total_ms / max(3, args.steps // 4)
 
     # Roofline of the dominant kernel (tcgen05 prefill): retained FLOPs only.
-    terms = atf.pruned_terms(N, D, base, kwin)
+    terms = atf.pruned_terms(N, D, base, kwin, **tk)
     flops = B * Hq * (4 * terms["kept"] + D * N * (N + 1))
     peaks, src = measured_peaks()
     long_region = total_ms > 2000.0
     peak = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
     achieved = flops / (kern_ms / 1e3) / 1e12
-    traffic = TRAFFIC["bytes_per_launch"] if TRAFFIC["source_sha1"] == kernel_sha1() else None
+    traffic = prefill_traffic(args.workload, wl)
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": f"prefill_tc_kernel<{D}>",
                 "kernel_ms": round(kern_ms, 4),
@@ -453,15 +533,44 @@ def run_decode(args, wl):
         kc = atf.rope_pack(kc.permute(0, 2, 1, 3).contiguous(), base)
         torch.cuda.synchronize()
     dkw = dict(kcache_rotated=True, kv_layout="PACKED") if packed else {}
+    page = wl.get("page")
+    if page:
+        # Cut the caches into pages and scatter them through one pool in a seeded
+        # random order (3 pool pages stay unused); built once, not timed.
+        import numpy as np
+        mp = L // page
+        n_pool = B * mp + 3
+        ids = np.random.default_rng(wl["seed"]).permutation(n_pool)[: B * mp].astype(np.int32)
+        bt = torch.as_tensor(ids.reshape(B, mp), device=dev)
+        idx = torch.as_tensor(ids.astype(np.int64), device=dev)
+        C = D // 16
+        if packed:  # [B*Hkv, C, L, 16] -> pool [n_pool, Hkv, C, page, 16]
+            kp = torch.zeros((n_pool, Hkv, C, page, 16), dtype=torch.bfloat16, device=dev)
+            kp[idx] = kc.view(B, Hkv, C, mp, page, 16).permute(0, 3, 1, 2, 4, 5).reshape(B * mp, Hkv, C, page, 16)
+        else:  # [B, Hkv, L, D] -> pool [n_pool, page, Hkv, D]
+            kp = torch.zeros((n_pool, page, Hkv, D), dtype=torch.bfloat16, device=dev)
+            kp[idx] = kc.view(B, Hkv, mp, page, D).permute(0, 2, 3, 1, 4).reshape(B * mp, page, Hkv, D)
+        vp = torch.zeros((n_pool, page, Hkv, D), dtype=torch.bfloat16, device=dev)
+        vp[idx] = vc.view(B, Hkv, mp, page, D).permute(0, 2, 3, 1, 4).reshape(B * mp, page, Hkv, D)
+        del kc, vc, idx
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        ws = torch.empty(atf.decode_workspace_bytes(B, Hq, Hkv, mp * page, D), dtype=torch.uint8, device=dev)
+
+        def call(kw):
+            atf.decode_paged(q, kp, vp, bt, sl, page, base, kw, out=out, workspace=ws, **dkw)
+    else:
+        def call(kw):
+            atf.decode(q, kc, vc, sl, base, kw, out=out, workspace=ws, **dkw)
 
     def timed(kw, steps):
         for _ in range(args.warmup):
-            atf.decode(q, kc, vc, sl, base, kw, out=out, workspace=ws, **dkw)
+            call(kw)
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(steps):
-            atf.decode(q, kc, vc, sl, base, kw, out=out, workspace=ws, **dkw)
+            call(kw)
         b.record(stream)
         torch.cuda.synchronize()
         return a.elapsed_time(b) / steps
@@ -472,8 +581,12 @@ def run_decode(args, wl):
     ms = timed(kwin, args.steps)
     clocks = sampler.stop()
     ms_off = timed(math.inf, args.steps)
+    if atf.device_status() != 0:
+        raise RuntimeError("a kernel's bounded wait ran out in the timed region")
     peaks, src = measured_peaks()
     nbytes = decode_retained_bytes(atf, wl)
+    if page:
+        nbytes += 4 * B * (L // page)  # the block table
     gbs = nbytes / (ms / 1e3) / 1e9
     line = {"metric": METRIC, "value": round(world * B / (ms / 1e3), 2), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
@@ -482,12 +595,153 @@ def run_decode(args, wl):
             "decode": {"us_per_call": round(1e3 * ms, 2), "us_per_token": round(1e3 * ms / B, 2)},
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": decode_traffic(args.workload, L),
-                         "kernel": f"decode_tc_kernel<{D}> + decode_merge_kernel",
+                         "kernel": f"decode_tc_kernel<{D}{', paged' if page else ''}> + decode_merge_kernel",
                          "bytes_per_call": nbytes, "peak_source": src},
             "window_off": {"ms_per_step": round(ms_off, 4), "us_per_token": round(1e3 * ms_off / B, 2)},
             "on_off_speedup": round(ms_off / ms, 4), "gpu_launches": 2 * args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def ragged_lengths(seed, total, lo, hi):
+    """Sequence lengths drawn log-uniform in [lo, hi] until they sum to `total` (the
+    last one cut to fit, so the batch also holds a short ragged tail)."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    out, left = [], total
+    while left > 0:
+        n = min(left, int(round(math.exp(rng.uniform(math.log(lo), math.log(hi))))))
+        out.append(n)
+        left -= n
+    return out
+
+
+def run_varlen(args, wl):
+    import torch
+    import long_context_attention_pair_b200 as atf
+    from long_context_attention_pair_b200 import synthetic
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    Hq, Hkv, D, base, kwin = wl["Hq"], wl["Hkv"], wl["D"], wl["rope_base"], wl["k_window"]
+    lens = ragged_lengths(wl["seed"], wl["total"], wl["len_lo"], wl["len_hi"])
+    total, max_len = sum(lens), max(lens)
+    cu_host = [0]
+    for n in lens:
+        cu_host.append(cu_host[-1] + n)
+    cu = torch.tensor(cu_host, dtype=torch.int32, device=dev)
+    q = synthetic.tensor_torch(wl["seed"], "q", (total, Hq, D), "bf16", device=dev)
+    k = synthetic.tensor_torch(wl["seed"], "k", (total, Hkv, D), "bf16", device=dev)
+    v = synthetic.tensor_torch(wl["seed"], "v", (total, Hkv, D), "bf16", device=dev)
+    out = torch.empty_like(q)
+    ws = torch.empty(int(atf.lib().atflash_prefill_varlen_workspace_bytes(Hq, Hkv, total, D)), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call(kw):
+        atf.prefill_varlen(q, k, v, cu, max_len, base, kw, out=out, workspace=ws)
+
+    def timed(kw, steps):
+        for _ in range(args.warmup):
+            call(kw)
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            call(kw)
+            b.record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    ms = timed(kwin, args.steps)
+    clocks = sampler.stop()
+    ms = reduce_max(ms, world, dev)
+    ms_off = reduce_max(timed(math.inf, args.steps), world, dev)
+    if atf.device_status() != 0:
+        raise RuntimeError("a kernel's bounded wait ran out in the timed region")
+
+    # Retained FLOPs: QK over the kept pair-terms of every sequence plus the causal PV.
+    flops = 0
+    kept = pruned = all_terms = 0
+    for n in lens:
+        t = atf.pruned_terms(n, D, base, kwin)
+        flops += Hq * (4 * t["kept"] + D * n * (n + 1))
+        kept, pruned, all_terms = kept + t["kept"], pruned + t["pruned"], all_terms + t["total"]
+    peaks, src = measured_peaks()
+    long_region = ms * args.steps > 2000.0
+    peak = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
+    achieved = flops / (ms / 1e3) / 1e12
+    line = {"metric": METRIC, "value": round(world * total / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(wl, B=len(lens), max_seqlen=max_len, seqlens=lens,
+                           l2="flushed before every step (256 MiB write, outside the timed events)"),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "kernel": f"whole call: rope_pack(q), rope_pack(k), prefill_tc_kernel<{D}, varlen>",
+                         "peak_source": f"{src} ({'sustained' if long_region else 'burst'} bf16)",
+                         "flops_per_launch": flops},
+            "window_off": {"ms_per_step": round(ms_off, 4), "value": round(world * total / (ms_off / 1e3), 1)},
+            "on_off_speedup": round(ms_off / ms, 4),
+            "pruned_fraction": round(pruned / all_terms, 6),
+            "gpu_launches": 3 * args.steps, "clocks": clocks}
+    if not args.no_e2e:
+        line["e2e"] = e2e_varlen(atf, q, k, v, cu, max_len, wl, args, dev, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n0 = lens[0]
+        line["cpu_baseline"] = cpu_baseline(q[None, :n0], k[None, :n0], v[None, :n0], dict(wl, N=n0))
+        line["cpu_baseline"]["sample"] += f" (first sequence of the batch, {n0} tokens)"
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def e2e_varlen(atf, q, k, v, cu, max_len, wl, args, dev, world):
+    """The ragged prefill through the public API with host buffers: every step copies
+    q/k/v/cu_seqlens from pinned host memory, runs the call and reads the output back,
+    all on one stream inside the timed region."""
+    import torch
+    hq, hk, hv, hcu = (t.cpu().pin_memory() for t in (q, k, v, cu))
+    hout = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv, dcu, dout = (torch.empty_like(t) for t in (q, k, v, cu, q))
+    ws = torch.empty(int(atf.lib().atflash_prefill_varlen_workspace_bytes(wl["Hq"], wl["Hkv"], q.shape[0],
+                                                                         wl["D"])), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    total = q.shape[0]
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dcu.copy_(hcu, non_blocking=True)
+        atf.prefill_varlen(dq, dk, dv, dcu, max_len, wl["rope_base"], wl["k_window"], out=dout, workspace=ws)
+        hout.copy_(dout, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    steps = max(3, args.steps)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = reduce_max(a.elapsed_time(b) / steps, world, dev)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcu))
+    return {"value": round(world * total / (ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": hout.numel() * hout.element_size(), "ms_per_step": round(ms, 4),
+            "api": "prefill_varlen"}
 
 
 def e2e(atf, q, k, v, wl, args, dev, world):
@@ -500,6 +754,8 @@ def e2e(atf, q, k, v, wl, args, dev, world):
     import torch
     B, N, Hq, Hkv, D = wl["B"], wl["N"], wl["Hq"], wl["Hkv"], wl["D"]
     base, kwin = wl["rope_base"], wl["k_window"]
+    th = rope_theta(wl)
+    tk = {} if th is None else {"theta": th}
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     hsl = torch.full((B,), N, dtype=torch.int32).pin_memory()
     nbuf = 2
@@ -538,10 +794,10 @@ def e2e(atf, q, k, v, wl, args, dev, world):
             s_comp.wait_event(in_done[bi])
             if used[bi]:
                 s_comp.wait_event(out_done[bi])  # step i-2's outputs have been read back
-            atf.prefill(d["q"], d["k"], d["v"], base, kwin, out=d["out"], workspace=d["ws"], stream=s_comp)
+            atf.prefill(d["q"], d["k"], d["v"], base, kwin, out=d["out"], workspace=d["ws"], stream=s_comp, **tk)
             d["qlast"].copy_(d["q"][:, N - 1])
             atf.decode(d["qlast"], d["k"], d["v"], d["sl"], base, kwin, kv_layout="NHD", out=d["dec"],
-                       workspace=d["dws"], stream=s_comp)
+                       workspace=d["dws"], stream=s_comp, **tk)
             comp_done[bi].record(s_comp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[bi])
@@ -580,6 +836,9 @@ def main():
         if args.k_window is not None:
             wl["k_window"] = args.k_window
         run_decode(args, wl)
+        return
+    if args.workload in VARLEN_WORKLOADS:
+        run_varlen(args, dict(VARLEN_WORKLOADS[args.workload]))
         return
     wl = dict(WORKLOADS[args.workload])
     if args.N:

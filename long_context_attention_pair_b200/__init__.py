@@ -85,12 +85,13 @@ def lib():
         L.atflash_prefill_varlen_theta.argtypes = [vp, vp, vp, vp, vp, i, i64, i64, i, i, i, dp, d, i, vp, vp, sz, vp]
         L.atflash_decode_paged_theta.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, dp, d, i, i, i, vp, sz,
                                                  vp]
+        L.atflash_prefill_packed_theta.argtypes = [vp, vp, vp, vp, i, i, i, i64, i, dp, d, i, i, vp, vp]
         for f in ("atflash_window_table", "atflash_pruned_terms", "atflash_prefill", "atflash_prefill_ex",
                   "atflash_decode", "atflash_device_status", "atflash_rope_pack", "atflash_prefill_packed",
                   "atflash_prefill_varlen", "atflash_decode_paged", "atflash_theta_table",
                   "atflash_window_table_theta", "atflash_pruned_terms_theta", "atflash_rope_pack_theta",
                   "atflash_prefill_theta", "atflash_decode_theta", "atflash_prefill_varlen_theta",
-                  "atflash_decode_paged_theta"):
+                  "atflash_decode_paged_theta", "atflash_prefill_packed_theta"):
             getattr(L, f).restype = i
         _lib = L
     return _lib
@@ -305,8 +306,9 @@ def rope_pack(x, rope_base: float, *, out=None, stream=None, theta=None):
 
 
 def prefill_packed(qpack, kpack, v, rope_base: float, k_window: float = math.inf, *, B=None, Hq=None,
-                   out=None, out_dtype=None, lse=None, stream=None):
-    """Attention over ``rope_pack`` outputs; v [B, N, Hkv, D] un-rotated values."""
+                   out=None, out_dtype=None, lse=None, stream=None, theta=None):
+    """Attention over ``rope_pack`` outputs; v [B, N, Hkv, D] un-rotated values.
+    With ``theta``, qpack/kpack come from ``rope_pack(..., theta=theta)``."""
     torch = _torch()
     Bv, N, Hkv, D = v.shape
     B = Bv if B is None else B
@@ -314,11 +316,13 @@ def prefill_packed(qpack, kpack, v, rope_base: float, k_window: float = math.inf
     if out is None:
         od = out_dtype if out_dtype is not None else v.dtype
         out = torch.empty((B, N, Hq, D), dtype=od, device=v.device)
-    st = lib().atflash_prefill_packed(_dev(qpack, "qpack"), _dev(kpack, "kpack"), _dev(v, "v"), _dev(out, "out"),
-                                      B, Hq, Hkv, N, D, float(rope_base), float(k_window), _dtype_code(v),
-                                      _dtype_code(out), _dev(lse, "lse") if lse is not None else None,
-                                      _stream_ptr(stream))
-    _check(st, "atflash_prefill_packed")
+    fn, name, rope = lib().atflash_prefill_packed, "atflash_prefill_packed", float(rope_base)
+    if theta is not None:
+        fn, name, rope = lib().atflash_prefill_packed_theta, "atflash_prefill_packed_theta", _theta_arg(theta, D)
+    st = fn(_dev(qpack, "qpack"), _dev(kpack, "kpack"), _dev(v, "v"), _dev(out, "out"), B, Hq, Hkv, N, D, rope,
+            float(k_window), _dtype_code(v), _dtype_code(out), _dev(lse, "lse") if lse is not None else None,
+            _stream_ptr(stream))
+    _check(st, name)
     return out
 
 

@@ -260,19 +260,34 @@ int atflash_rope_pack_theta(const void *x, void *y, int B, int64_t N, int H, int
     return rope_pack_impl(x, y, B, N, H, D, theta, in_dtype, stream);
 }
 
+static int prefill_packed_impl(const void *qpack, const void *kpack, const void *v, void *out, int B, int Hq,
+                               int Hkv, int64_t N, int D, const double *theta, double k_window, int in_dtype,
+                               int out_dtype, float *lse, cudaStream_t stream) {
+    int rc = check_prefill_common(B, Hq, Hkv, N, D, theta, k_window, in_dtype, out_dtype);
+    if (rc != ATFLASH_OK) return rc;
+    if ((reinterpret_cast<uintptr_t>(qpack) & 255u) || (reinterpret_cast<uintptr_t>(kpack) & 255u) ||
+        !aligned16(v) || !aligned16(out))
+        return ATFLASH_ERR_ALIGNMENT;
+    return run_prefill_packed(qpack, kpack, v, out, B, Hq, Hkv, N, D, theta, k_window, in_dtype, out_dtype, lse,
+                              stream);
+}
+
 int atflash_prefill_packed(const void *qpack, const void *kpack, const void *v, void *out, int B, int Hq,
                            int Hkv, int64_t N, int D, double rope_base, double k_window, int in_dtype,
                            int out_dtype, float *lse, cudaStream_t stream) {
     if (!qpack || !kpack || !v || !out) return ATFLASH_ERR_INVALID_ARG;
     BaseTheta bt(D, rope_base);
     if (bt.rc != ATFLASH_OK) return bt.rc;
-    int rc = check_prefill_common(B, Hq, Hkv, N, D, bt.theta, k_window, in_dtype, out_dtype);
-    if (rc != ATFLASH_OK) return rc;
-    if ((reinterpret_cast<uintptr_t>(qpack) & 255u) || (reinterpret_cast<uintptr_t>(kpack) & 255u) ||
-        !aligned16(v) || !aligned16(out))
-        return ATFLASH_ERR_ALIGNMENT;
-    return run_prefill_packed(qpack, kpack, v, out, B, Hq, Hkv, N, D, bt.theta, k_window, in_dtype, out_dtype,
-                              lse, stream);
+    return prefill_packed_impl(qpack, kpack, v, out, B, Hq, Hkv, N, D, bt.theta, k_window, in_dtype, out_dtype,
+                               lse, stream);
+}
+
+int atflash_prefill_packed_theta(const void *qpack, const void *kpack, const void *v, void *out, int B, int Hq,
+                                 int Hkv, int64_t N, int D, const double *theta, double k_window, int in_dtype,
+                                 int out_dtype, float *lse, cudaStream_t stream) {
+    if (!qpack || !kpack || !v || !out) return ATFLASH_ERR_INVALID_ARG;
+    return prefill_packed_impl(qpack, kpack, v, out, B, Hq, Hkv, N, D, theta, k_window, in_dtype, out_dtype, lse,
+                               stream);
 }
 
 static int prefill_ex_impl(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,

@@ -28,8 +28,10 @@
 // chunk.  A pruned chunk of 64 keys is then 2 KB of HBM that is never fetched.
 // In the natural layouts a key's pruned dims are a prefix of each half-row; the
 // copy fetches each half in 32-byte (16-dim) boxes from the first 32-byte sector
-// that some key of the stage keeps, the finest cut that saves DRAM traffic (the
-// DRAM sector is 32 bytes).  The 2 KB of one chunk
+// that some key of the stage keeps.  That saves shared-memory fills and consumer
+// work but no DRAM traffic: every half-row keeps its lowest-frequency sector, and
+// the memory system brings a 128-byte half-row in whole once any of its sectors
+// is read (measured: the whole cache per launch).  The 2 KB of one chunk
 // of a stage are contiguous, so the copy views them as 16 rows of 128 bytes
 // (4 keys per row, SWIZZLE_128B) rather than 64 rows of 32 bytes: a quarter of
 // the TMA row requests, which bound the producer otherwise.  That view needs

@@ -270,8 +270,12 @@ def test_theta_tables_rejected(L):
                                               1 << 40, None) == -1, name
         assert L.atflash_decode_paged_theta(P, P, P, P, P, P, 1, 2, 1, 4, 8, 64, 64, arr, 1.0, 0, atf.KV_NHD,
                                             atf.F32, P, 1 << 40, None) == -1, name
+        assert L.atflash_prefill_packed_theta(P, P, P, P, 1, 2, 1, 256, 64, arr, 1.0, atf.BF16, atf.BF16, None,
+                                              None) == -1, name
     assert L.atflash_prefill_theta(P, P, P, P, 1, 2, 1, 256, 64, None, 1.0, atf.BF16, atf.BF16, None, P,
                                    1 << 40, None) == -1
+    assert L.atflash_prefill_packed_theta(P, P, P, P, 1, 2, 1, 256, 64, None, 1.0, atf.BF16, atf.BF16, None,
+                                          None) == -1
     assert L.atflash_theta_table(64, 1.0, (ctypes.c_double * 32)()) == -1
     with pytest.raises(ValueError):
         atf.window_table(64, 0.0, 1.0, 100, theta=good[:-1])

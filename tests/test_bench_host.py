@@ -1,0 +1,61 @@
+"""Host-side checks of the benchmark's workload tables (no GPU)."""
+import math
+
+import bench
+
+
+def test_ragged_lengths_fill_the_total_within_bounds():
+    for wl in bench.VARLEN_WORKLOADS.values():
+        lens = bench.ragged_lengths(wl["seed"], wl["total"], wl["len_lo"], wl["len_hi"])
+        assert sum(lens) == wl["total"]
+        assert all(1 <= n <= wl["len_hi"] for n in lens)
+        # every length but the cut last one lies in [lo, hi]
+        assert all(n >= wl["len_lo"] for n in lens[:-1])
+        assert len(set(lens)) > 1  # ragged, not uniform
+        assert lens == bench.ragged_lengths(wl["seed"], wl["total"], wl["len_lo"], wl["len_hi"])
+
+
+def test_paged_workloads_split_into_whole_pages():
+    for name, wl in bench.DECODE_WORKLOADS.items():
+        if "page" in wl:
+            assert wl["page"] % 64 == 0 and wl["N"] % wl["page"] == 0, name
+
+
+def test_workload_names_are_unique_across_tables():
+    names = list(bench.WORKLOADS) + list(bench.DECODE_WORKLOADS) + list(bench.VARLEN_WORKLOADS)
+    assert len(names) == len(set(names))
+    assert all(math.isfinite(w["k_window"]) for w in bench.VARLEN_WORKLOADS.values())
+
+
+def test_scaled_workload_theta_is_the_llama3_table():
+    import numpy as np
+    from scaled import llama3_scaled_theta
+    for name in ("llama3b_128k_scaled",):
+        wl = bench.WORKLOADS[name]
+        sc = wl["rope_scaling"]
+        th = np.array(bench.rope_theta(wl))
+        ref = llama3_scaled_theta(wl["D"], wl["rope_base"], factor=sc["factor"], low=sc["low_freq_factor"],
+                                  high=sc["high_freq_factor"], orig_ctx=sc["original_max_position_embeddings"])
+        np.testing.assert_allclose(th, ref, rtol=1e-13, atol=0)
+        assert np.all(np.diff(th) <= 0) and th[0] <= math.pi and th[-1] > 0
+        assert bench.rope_theta(bench.WORKLOADS["llama3b_32k"]) is None
+
+
+def test_scaled_workload_table_is_accepted_by_the_library():
+    import long_context_attention_pair_b200 as atf
+    wl = bench.WORKLOADS["llama3b_128k_scaled"]
+    th = bench.rope_theta(wl)
+    w = atf.window_table(wl["D"], 0.0, wl["k_window"], wl["N"], theta=th)
+    w0 = atf.window_table(wl["D"], wl["rope_base"], wl["k_window"], wl["N"])
+    # scaling divides the low frequencies: their windows only grow
+    assert all(a >= b for a, b in zip(w, w0)) and w != w0
+
+
+def test_captured_traffic_is_reported_only_for_its_own_workload():
+    wl = dict(bench.WORKLOADS["qwen05b_32k"])
+    same_source = bench.TRAFFIC["source_sha1"] == bench.kernel_sha1()
+    assert (bench.prefill_traffic("qwen05b_32k", wl) is not None) == same_source
+    assert bench.prefill_traffic("llama3b_128k", dict(bench.WORKLOADS["llama3b_128k"])) is None
+    assert bench.prefill_traffic("qwen05b_32k", dict(wl, N=65536)) is None
+    assert bench.prefill_traffic("qwen05b_32k", dict(wl, k_window=float("inf"))) is None
+    assert bench.decode_traffic("decode_128k", 1 << 17) is None
