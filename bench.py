@@ -144,10 +144,10 @@ TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 99188992,
 # the full-size workloads, from single-pass ncu captures
 # (profiles/decode_tc_qwen7b_packed_4x128k.md); valid while decode_tc.cu hashes to
 # `source_sha1`.
-DECODE_TRAFFIC = {"decode_1m_packed": {"bytes_per_launch": 6607405312,
-                                       "source_sha1": "d7b5169d59996c1a554d660578c2ccb20b0d7d15"},
-                  "decode_1m": {"bytes_per_launch": 8608839424,
-                                "source_sha1": "d7b5169d59996c1a554d660578c2ccb20b0d7d15"}}
+DECODE_TRAFFIC = {"decode_1m_packed": {"bytes_per_launch": 6607293952,
+                                       "source_sha1": "61a5dcf9b9fce74f5022cf838de7d70f2150435d"},
+                  "decode_1m": {"bytes_per_launch": 8608907008,
+                                "source_sha1": "61a5dcf9b9fce74f5022cf838de7d70f2150435d"}}
 
 
 def parse():

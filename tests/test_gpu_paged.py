@@ -120,3 +120,39 @@ def test_paged_bad_page_ids_read_zeros_without_fault():
     torch.cuda.synchronize()
     assert atf.device_status() == 0
     assert torch.isfinite(out).all()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("packed", [True, False])
+def test_paged_bench_size_equals_contiguous(packed):
+    # The benchmark's paged workload (4 x 1M keys of the Qwen2.5-7B-1M shape in
+    # shuffled 256-token pages): bit-identical to the contiguous cache, whose
+    # full-size parity against the oracle the decode tests check.
+    B, Hq, Hkv, L, D, P_, base, kwin = 4, 28, 4, 1 << 20, 128, 256, 1e7, 16.0
+    q = P.gen(77, "q_dec", (B, Hq, D), "bf16")
+    kc = P.gen(77, "k_cache", (B, Hkv, L, D), "bf16")
+    vc = P.gen(77, "v_cache", (B, Hkv, L, D), "bf16")
+    sl = torch.full((B,), L, dtype=torch.int32, device="cuda")
+    mp = L // P_
+    ids, n_pool = scatter_pages(B, Hkv, L, P_, 78)
+    idx = torch.as_tensor(ids.reshape(-1).astype(np.int64), device="cuda")
+    C = D // 16
+    vp = torch.zeros((n_pool, P_, Hkv, D), dtype=vc.dtype, device="cuda")
+    vp[idx] = vc.view(B, Hkv, mp, P_, D).permute(0, 2, 3, 1, 4).reshape(B * mp, P_, Hkv, D)
+    if packed:
+        kcont = atf.rope_pack(kc.permute(0, 2, 1, 3).contiguous(), base)
+        kp = torch.zeros((n_pool, Hkv, C, P_, 16), dtype=kc.dtype, device="cuda")
+        kp[idx] = kcont.view(B, Hkv, C, mp, P_, 16).permute(0, 3, 1, 2, 4, 5).reshape(B * mp, Hkv, C, P_, 16)
+        kw = dict(kcache_rotated=True, kv_layout="PACKED")
+    else:
+        kcont = kc
+        kp = torch.zeros((n_pool, P_, Hkv, D), dtype=kc.dtype, device="cuda")
+        kp[idx] = kc.view(B, Hkv, mp, P_, D).permute(0, 2, 3, 1, 4).reshape(B * mp, P_, Hkv, D)
+        kw = {}
+    bt = torch.as_tensor(ids, device="cuda")
+    out = atf.decode_paged(q, kp, vp, bt, sl, P_, base, kwin, kv_layout=kw.get("kv_layout", "NHD"),
+                           kcache_rotated=kw.get("kcache_rotated", False))
+    ref = atf.decode(q, kcont, vc, sl, base, kwin, **kw)
+    torch.cuda.synchronize()
+    assert atf.device_status() == 0
+    assert torch.equal(out, ref)

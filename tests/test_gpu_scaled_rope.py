@@ -142,3 +142,24 @@ def test_scaled_paged_decode_equals_contiguous_scaled_decode():
     torch.cuda.synchronize()
     assert atf.device_status() == 0
     assert torch.equal(out, ref)
+
+
+@pytest.mark.slow
+def test_scaled_prefill_llama3b_128k_sampled(oracle):
+    # The benchmark's scaled-RoPE workload (Llama-3.2-3B shape with its llama3
+    # rope_scaling table at 128K), sampled query rows of every head.
+    import bench
+    wl = bench.WORKLOADS["llama3b_128k_scaled"]
+    th = bench.rope_theta(wl)
+    N, Hq, Hkv, D, kwin = wl["N"], wl["Hq"], wl["Hkv"], wl["D"], wl["k_window"]
+    q = P.gen(76, "q", (1, N, Hq, D), "bf16")
+    k = P.gen(76, "k", (1, N, Hkv, D), "bf16")
+    v = P.gen(76, "v", (1, N, Hkv, D), "bf16")
+    out = atf.prefill(q, k, v, 0.0, kwin, theta=th)
+    torch.cuda.synchronize()
+    assert atf.device_status() == 0
+    rows = P.sample_rows(N, 24, 76)
+    idx = torch.as_tensor(rows, device=q.device)
+    with oracle.scaled_rope(th):
+        ref = oracle.prefill_rows(P.host(q[0, idx]), rows, P.host(k[0]), P.host(v[0]), wl["rope_base"], kwin)
+    P.check(P.host(out[0, idx]), ref, "bf16", "scaled 128K")

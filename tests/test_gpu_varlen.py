@@ -88,3 +88,21 @@ def test_varlen_malformed_table_leaves_those_rows_untouched(oracle):
     assert atf.device_status() == 0
     assert torch.all(out[200:] == 7.0)
     check_against_oracle(oracle, q, k, v, cu[:2], out, base, kwin)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,rows", [("varlen_qwen05b_256k", 16), ("varlen_qwen7b_1m", 6)])
+def test_varlen_bench_mix_sampled(oracle, name, rows):
+    # The benchmark's ragged batches, in its launch configuration (bf16 out,
+    # caller's workspace): sampled rows of every sequence against the oracle.
+    import bench
+    wl = bench.VARLEN_WORKLOADS[name]
+    lens = bench.ragged_lengths(wl["seed"], wl["total"], wl["len_lo"], wl["len_hi"])
+    q, k, v, cu = packed_batch(64, lens, wl["Hq"], wl["Hkv"], wl["D"])
+    ws = torch.empty(int(atf.lib().atflash_prefill_varlen_workspace_bytes(wl["Hq"], wl["Hkv"], q.shape[0], wl["D"])),
+                     dtype=torch.uint8, device="cuda")
+    out = atf.prefill_varlen(q, k, v, torch.as_tensor(cu, device="cuda"), max(lens), wl["rope_base"],
+                             wl["k_window"], workspace=ws)
+    torch.cuda.synchronize()
+    assert atf.device_status() == 0
+    check_against_oracle(oracle, q, k, v, cu, out, wl["rope_base"], wl["k_window"], max_rows=rows, seed=65)
