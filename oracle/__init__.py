@@ -44,6 +44,9 @@ def lib():
         L.orc_min_kept_pairs.restype = i64
         L.orc_prefill_rows.argtypes = [fp, i64p, i64, fp, fp, i, i, i64, i, d, d, dp, dp]
         L.orc_prefill_rows.restype = i
+        L.orc_prefill_rows_sparse.argtypes = [fp, i64p, i64, fp, fp, i, i, i64, i, d, d,
+                                              ctypes.POINTER(ctypes.c_ubyte), i64, dp, dp]
+        L.orc_prefill_rows_sparse.restype = i
         L.orc_decode.argtypes = [fp, fp, fp, i32p, i, i, i, i64, i, d, d, i, dp, dp]
         L.orc_decode.restype = i
         L.orc_rope_rows.argtypes = [fp, i64p, i64, i, d, dp]
@@ -149,6 +152,30 @@ def prefill_rows(q_rows, rows, k, v, base: float, kwin: float, want_lse: bool = 
                                 base, kwin, _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
     if rc != 0:
         raise ValueError("oracle prefill_rows rejected its arguments")
+    return (out, lse) if want_lse else out
+
+
+def prefill_rows_sparse(q_rows, rows, k, v, base: float, kwin: float, block_mask, tile: int = 128,
+                        want_lse: bool = False):
+    """prefill_rows under a token-level block selection: block_mask [Hkv, T, T]
+    (T = ceil(N / tile)); key m is visible to query n iff m <= n and (same tile,
+    or block_mask[g, n // tile, m // tile] != 0) for the query heads of KV head g."""
+    q_rows, k, v = _f32(q_rows), _f32(k), _f32(v)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    R, Hq, D = q_rows.shape
+    N, Hkv, _ = k.shape
+    T = (N + tile - 1) // tile
+    mask = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
+    if mask.shape != (Hkv, T, T):
+        raise ValueError(f"block_mask must be [{Hkv}, {T}, {T}]")
+    out = np.zeros((R, Hq, D), dtype=np.float64)
+    lse = np.zeros((R, Hq), dtype=np.float64)
+    rc = lib().orc_prefill_rows_sparse(_ptr(q_rows, ctypes.c_float), _ptr(rows, ctypes.c_int64), R,
+                                       _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float), Hq, Hkv, N, D,
+                                       base, kwin, _ptr(mask, ctypes.c_ubyte), tile,
+                                       _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise ValueError("oracle prefill_rows_sparse rejected its arguments")
     return (out, lse) if want_lse else out
 
 

@@ -25,6 +25,15 @@
  * unchanged.  (The pages derive the window table from the model's RoPE
  * configuration, "rope_scaling" included.)
  *
+ * Token-level selection under the window (the abstract: token-level sparse
+ * methods such as MInference are orthogonal to the frequency-level window, which
+ * can be applied on top of them): orc_prefill_rows_sparse takes a block mask
+ * over (query tile, key tile) pairs of `tile` positions each.  Key m is visible
+ * to query n iff m <= n and (m and n lie in the same tile, or the mask entry of
+ * their tiles is nonzero); the diagonal tile is always visible, so no row is
+ * empty.  Invisible keys take no part in the softmax; the window applies to the
+ * visible ones unchanged.
+ *
  * k = +inf keeps every pair (plain causal RoPE attention).  A cell whose every
  * pair is pruned scores 0 (the empty sum), not -inf: the pages keep "the sum
  * over the rest" and drop no token.
@@ -162,18 +171,29 @@ static double orc_score(const double *qt, const double *kt, int D, const double 
     return acc / sqrt((double)D);
 }
 
-/* Attention output of one query row over keys 0..n (rotated keys kt[m*D..]),
- * two-pass softmax.  out[D]; *lse = natural log-sum-exp of the scores. */
+/* Is key m visible to query n under the block mask row of n's tile (NULL: all
+ * keys 0..n are)? */
+static int orc_visible(const unsigned char *mask_row, int64_t tile, int64_t n, int64_t m) {
+    if (!mask_row) return 1;
+    return m / tile == n / tile || mask_row[m / tile] != 0;
+}
+
+/* Attention output of one query row over the visible keys among 0..n (rotated
+ * keys kt[m*D..]), two-pass softmax.  out[D]; *lse = natural log-sum-exp of the
+ * scores. */
 static void orc_row(const double *qt, const double *kt, const float *v, int64_t v_stride,
-                    int64_t n, int D, const double *lim, double *scores, double *out, double *lse) {
+                    int64_t n, int D, const double *lim, const unsigned char *mask_row, int64_t tile,
+                    double *scores, double *out, double *lse) {
     double mx = -INFINITY;
     for (int64_t m = 0; m <= n; ++m) {
+        if (!orc_visible(mask_row, tile, n, m)) continue;
         scores[m] = orc_score(qt, kt + (size_t)m * D, D, lim, n - m);
         if (scores[m] > mx) mx = scores[m];
     }
     double den = 0.0;
     for (int i = 0; i < D; ++i) out[i] = 0.0;
     for (int64_t m = 0; m <= n; ++m) {
+        if (!orc_visible(mask_row, tile, n, m)) continue;
         double p = exp(scores[m] - mx);
         den += p;
         const float *vm = v + (size_t)m * (size_t)v_stride;
@@ -205,10 +225,13 @@ static double *orc_rotated_keys(const float *k, int64_t k_stride, int64_t nk, in
  *   out    [nrows][Hq][D], lse [nrows][Hq] (lse may be NULL)
  * Query head h reads KV head h / (Hq / Hkv).  Returns 0, or -1 on bad input.
  */
-int orc_prefill_rows(const float *q_rows, const int64_t *rows, int64_t nrows,
-                     const float *k, const float *v, int Hq, int Hkv, int64_t N, int D,
-                     double base, double kwin, double *out, double *lse) {
+static int orc_prefill_rows_masked(const float *q_rows, const int64_t *rows, int64_t nrows,
+                                   const float *k, const float *v, int Hq, int Hkv, int64_t N, int D,
+                                   double base, double kwin, const unsigned char *block_mask, int64_t tile,
+                                   double *out, double *lse) {
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || D % 2 || N <= 0) return -1;
+    if (block_mask && tile <= 0) return -1;
+    int64_t ntiles = block_mask ? (N + tile - 1) / tile : 0;
     int G = Hq / Hkv;
     int H = D / 2;
     int64_t nmax = 0;
@@ -233,8 +256,10 @@ int orc_prefill_rows(const float *q_rows, const int64_t *rows, int64_t nrows,
                 int64_t i = t / G;
                 int h = g * G + (int)(t % G);
                 int64_t n = rows[i];
+                const unsigned char *mrow =
+                    block_mask ? block_mask + ((size_t)g * ntiles + (size_t)(n / tile)) * (size_t)ntiles : NULL;
                 orc_rope(q_rows + ((size_t)i * Hq + h) * D, D, base, n, qt);
-                orc_row(qt, kt, vg, (int64_t)Hkv * D, n, D, lim, scores,
+                orc_row(qt, kt, vg, (int64_t)Hkv * D, n, D, lim, mrow, tile, scores,
                         out + ((size_t)i * Hq + h) * D,
                         lse ? lse + (size_t)i * Hq + h : NULL);
             }
@@ -245,6 +270,28 @@ int orc_prefill_rows(const float *q_rows, const int64_t *rows, int64_t nrows,
     }
     free(lim);
     return rc;
+}
+
+int orc_prefill_rows(const float *q_rows, const int64_t *rows, int64_t nrows,
+                     const float *k, const float *v, int Hq, int Hkv, int64_t N, int D,
+                     double base, double kwin, double *out, double *lse) {
+    return orc_prefill_rows_masked(q_rows, rows, nrows, k, v, Hq, Hkv, N, D, base, kwin, NULL, 0, out, lse);
+}
+
+/*
+ * The same under a token-level block selection: block_mask [Hkv][T][T] with
+ * T = ceil(N / tile); entry (g, i, j) != 0 makes key tile j visible to query
+ * tile i for the query heads of KV head g (entries j > i only ever cover keys
+ * past the query and so change nothing; the diagonal entry is ignored: the
+ * diagonal tile is always visible).
+ */
+int orc_prefill_rows_sparse(const float *q_rows, const int64_t *rows, int64_t nrows,
+                            const float *k, const float *v, int Hq, int Hkv, int64_t N, int D,
+                            double base, double kwin, const unsigned char *block_mask, int64_t tile,
+                            double *out, double *lse) {
+    if (!block_mask) return -1;
+    return orc_prefill_rows_masked(q_rows, rows, nrows, k, v, Hq, Hkv, N, D, base, kwin, block_mask, tile, out,
+                                   lse);
 }
 
 /*
@@ -275,7 +322,7 @@ int orc_decode(const float *q, const float *kcache, const float *vcache, const i
             for (int j = 0; j < G; ++j) {
                 int h = g * G + j;
                 orc_rope(q + ((size_t)b * Hq + h) * D, D, base, L - 1, qt);
-                orc_row(qt, kt, vcache + base_off, D, L - 1, D, lim, scores,
+                orc_row(qt, kt, vcache + base_off, D, L - 1, D, lim, NULL, 0, scores,
                         out + ((size_t)b * Hq + h) * D, lse ? lse + (size_t)b * Hq + h : NULL);
             }
             free(scores);

@@ -328,3 +328,81 @@ def test_scaled_decode_equals_prefill_last_row(oracle):
         pre = oracle.prefill(q, k, v, base, 0.5)
         dec = oracle.decode(q[:, N - 1], k.transpose(0, 2, 1, 3), v.transpose(0, 2, 1, 3), [N], base, 0.5)
     np.testing.assert_allclose(dec, pre[:, N - 1], rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------- token-level block selection under the window
+def visible_textbook(N, tile, mask_g):
+    """Boolean [N, N]: key m visible to query n (causal, same tile, or mask entry set)."""
+    n = np.arange(N)[:, None]
+    m = np.arange(N)[None, :]
+    return (m <= n) & ((m // tile == n // tile) | (mask_g[n // tile, m // tile] != 0))
+
+
+def masked_attention_textbook(s, vis, v):
+    s = np.where(vis, s, -np.inf)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ np.asarray(v, dtype=np.float64)
+
+
+def random_block_mask(Hkv, T, seed, density=0.4):
+    rng = np.random.default_rng(seed)
+    return (rng.random((Hkv, T, T)) < density).astype(np.uint8)
+
+
+@pytest.mark.parametrize("kwin", [math.inf, 1.0])
+def test_sparse_equals_textbook_masked_softmax(oracle, kwin):
+    # Softmax over the visible keys only, written out with numpy from the score
+    # matrix: RoPE in matrix form for k = inf, the oracle's windowed scores
+    # (pinned above) otherwise.  Two KV groups with different masks.
+    N, D, Hq, Hkv, tile, base = 70, 16, 4, 2, 16, 1e4
+    T = (N + tile - 1) // tile
+    q, k, v = rand((N, Hq, D), 81), rand((N, Hkv, D), 82, "k"), rand((N, Hkv, D), 83, "v")
+    mask = random_block_mask(Hkv, T, 84)
+    out = oracle.prefill_rows_sparse(q, np.arange(N), k, v, base, kwin, mask, tile)
+    G = Hq // Hkv
+    for h in range(Hq):
+        g = h // G
+        if math.isinf(kwin):
+            pos = np.arange(N)
+            s = rope_textbook(q[:, h], pos, base) @ rope_textbook(k[:, g], pos, base).T / math.sqrt(D)
+        else:
+            s = oracle.scores(q[:, h], k[:, g], base, kwin)
+        ref = masked_attention_textbook(s, visible_textbook(N, tile, mask[g]), v[:, g])
+        np.testing.assert_allclose(out[:, h], ref, rtol=0, atol=1e-12)
+
+
+def test_sparse_all_visible_equals_dense(oracle):
+    N, D, Hq, Hkv, tile, base = 90, 32, 2, 1, 16, 1e4
+    T = (N + tile - 1) // tile
+    q, k, v = rand((N, Hq, D), 85), rand((N, Hkv, D), 86, "k"), rand((N, Hkv, D), 87, "v")
+    rows = np.arange(N)
+    dense = oracle.prefill_rows(q, rows, k, v, base, 2.0)
+    sparse = oracle.prefill_rows_sparse(q, rows, k, v, base, 2.0, np.ones((Hkv, T, T), np.uint8), tile)
+    assert np.array_equal(dense, sparse)
+
+
+def test_sparse_diagonal_and_future_entries_are_ignored(oracle):
+    # The diagonal tile is always visible and entries above it cover only future
+    # keys: zeroing the diagonal and setting every entry above it changes nothing.
+    N, D, Hq, Hkv, tile, base = 64, 16, 2, 2, 8, 1e4
+    T = N // tile
+    q, k, v = rand((N, Hq, D), 88), rand((N, Hkv, D), 89, "k"), rand((N, Hkv, D), 90, "v")
+    mask = random_block_mask(Hkv, T, 91)
+    a_mask = mask.copy()
+    for g in range(Hkv):
+        a_mask[g] = np.tril(a_mask[g], -1) + np.eye(T, dtype=np.uint8)
+    b_mask = mask.copy()
+    for g in range(Hkv):
+        b_mask[g] = np.tril(b_mask[g], -1) + np.triu(np.ones((T, T), np.uint8), 1)
+    rows = np.arange(N)
+    a = oracle.prefill_rows_sparse(q, rows, k, v, base, 1.0, a_mask, tile)
+    b = oracle.prefill_rows_sparse(q, rows, k, v, base, 1.0, b_mask, tile)
+    assert np.array_equal(a, b)
+    # a query sees exactly its own tile's causal prefix when only the diagonal is set
+    only_diag = oracle.prefill_rows_sparse(q, rows, k, v, base, math.inf, np.zeros((Hkv, T, T), np.uint8), tile)
+    n = 21  # tile 2 (positions 16..23): keys 16..21
+    ref = attention_textbook(q[16:n + 1, 0], k[16:n + 1, 0], v[16:n + 1, 0], base)[-1]
+    # the textbook attention above starts positions at 0; RoPE scores depend on n - m only
+    np.testing.assert_allclose(only_diag[n, 0], ref, rtol=0, atol=1e-12)

@@ -2,11 +2,12 @@
 
 Each case copies the oracle to a temporary directory, plants one mistake in the
 copied C source (a wrong comparison, sign, index, scale, exponent, count term,
-empty-sum reading or decode position), builds it, and runs the pin tests of
+empty-sum reading, decode position or block-selection rule), builds it, and runs the pin tests of
 ``test_oracle.py`` against the copy: at least one pin must fail.  Mistakes are
 only ever planted in these CPU copies.
 """
 import importlib.util
+import math
 import os
 import shutil
 import sys
@@ -30,6 +31,12 @@ MUTANTS = {
                                "return acc == 0.0 ? -INFINITY : acc / sqrt((double)D);"),
     "decode_position": ("orc_rope(q + ((size_t)b * Hq + h) * D, D, base, L - 1, qt);",
                         "orc_rope(q + ((size_t)b * Hq + h) * D, D, base, L, qt);"),
+    "sparse_diagonal_not_forced": ("return m / tile == n / tile || mask_row[m / tile] != 0;",
+                                   "return mask_row[m / tile] != 0;"),
+    "sparse_group_index": ("block_mask ? block_mask + ((size_t)g * ntiles",
+                           "block_mask ? block_mask + ((size_t)0 * ntiles"),
+    "sparse_query_tile": ("+ (size_t)(n / tile)) * (size_t)ntiles : NULL;",
+                          "+ (size_t)(n / tile + 1) % ntiles) * (size_t)ntiles : NULL;"),
 }
 
 PIN_TESTS = [
@@ -45,6 +52,8 @@ PIN_TESTS = [
     lambda o: pins.test_k_zero_closed_form(o),
     lambda o: pins.test_single_pair_window_bruteforce(o),
     lambda o: pins.test_decode_equals_prefill_last_row(o),
+    lambda o: [pins.test_sparse_equals_textbook_masked_softmax(o, kw) for kw in (math.inf, 1.0)],
+    lambda o: pins.test_sparse_diagonal_and_future_entries_are_ignored(o),
 ]
 
 
