@@ -119,6 +119,136 @@ DECODE_WORKLOADS = {
                         "(256-token pages, shuffled pool)", "B": 4, "Hq": 28, "Hkv": 4, "D": 128, "N": 1 << 20,
                         "rope_base": 1e7, "k_window": 16.0, "seed": 4, "page": 256},
 }
+# Block-selected prefill workloads (the window on top of a token-level selection):
+# one step = one atflash_prefill_sparse call (RoPE pre-pass of Q and K, then the
+# windowed prefill over the selected 128 x 128 tiles).  The mask follows the shape
+# of dynamic-sparse selections such as MInference's: the first `sink_tiles` key
+# tiles of every query tile, a band of `local_tiles` tiles ending at the diagonal,
+# and each remaining causal tile with probability `extra` (seeded), per KV head.
+SPARSE_WORKLOADS = {
+    "qwen05b_32k_sparse": dict(_pf("Qwen2.5-0.5B-shaped single-layer windowed prefill over a block-sparse selection",
+                                   1, 14, 2, 64, 32768, 1e6, 8.0, 1),
+                               sink_tiles=2, local_tiles=16, extra=0.05, mask_seed=8),
+    "llama3b_128k_sparse": dict(_pf("Llama-3.2-3B-shaped single-layer windowed prefill over a block-sparse selection",
+                                    1, 24, 8, 128, 131072, 5e5, 16.0, 2),
+                                sink_tiles=2, local_tiles=32, extra=0.02, mask_seed=9),
+}
+
+
+def block_mask_recipe(wl, T):
+    """uint8 [B, Hkv, T, T] block selection of a SPARSE_WORKLOADS entry."""
+    import numpy as np
+    rng = np.random.default_rng(wl["mask_seed"])
+    m = rng.random((wl["B"], wl["Hkv"], T, T)) < wl["extra"]
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    m |= (j < wl["sink_tiles"]) | ((i - j >= 0) & (i - j < wl["local_tiles"]))
+    m &= j <= i
+    return m.astype(np.uint8)
+
+
+def tile_retained_flops(atf, wl, T):
+    """Retained FLOPs of one (query tile, key tile) pair of one query head, by
+    tile distance t = i - j: 4 per kept pair-term (QK over the kept pairs of each
+    cell) + 2*D per cell (PV).  N must be a multiple of 128."""
+    import numpy as np
+    D, N = wl["D"], wl["N"]
+    w = np.array(atf.window_table(D, wl["rope_base"], wl["k_window"], N), dtype=np.int64)
+    ws = np.sort(w)
+    kept_at = lambda d: len(ws) - np.searchsorted(ws, d, side="left")  # noqa: E731  pairs with w_r >= d
+    out = np.zeros(T, dtype=np.float64)
+    delta = np.arange(-127, 128)
+    mult = 128 - np.abs(delta)
+    for t in range(T):
+        if t == 0:
+            d = np.arange(128)
+            cnt = 128 - d                      # cells (a, b) with a - b = d, a >= b
+            kept = float(np.sum(cnt * kept_at(d)))
+            cells = 128 * 129 / 2
+        else:
+            d = 128 * t + delta
+            kept = float(np.sum(mult * kept_at(d)))
+            cells = 128 * 128
+        out[t] = 4 * kept + 2 * D * cells
+    return out
+
+
+def run_sparse(args, wl):
+    import numpy as np
+    import torch
+    import long_context_attention_pair_b200 as atf
+    from long_context_attention_pair_b200 import synthetic
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, N, Hq, Hkv, D = wl["B"], wl["N"], wl["Hq"], wl["Hkv"], wl["D"]
+    base, kwin = wl["rope_base"], wl["k_window"]
+    T = (N + 127) // 128
+    mask_np = block_mask_recipe(wl, T)
+    mask = torch.as_tensor(mask_np, device=dev)
+    q = synthetic.tensor_torch(wl["seed"], "q", (B, N, Hq, D), "bf16", device=dev)
+    k = synthetic.tensor_torch(wl["seed"], "k", (B, N, Hkv, D), "bf16", device=dev)
+    v = synthetic.tensor_torch(wl["seed"], "v", (B, N, Hkv, D), "bf16", device=dev)
+    out = torch.empty_like(q)
+    ws = torch.empty(atf.prefill_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    sparse_on = lambda: atf.prefill_sparse(q, k, v, mask, base, kwin, out=out, workspace=ws)  # noqa: E731
+    sparse_off = lambda: atf.prefill_sparse(q, k, v, mask, base, math.inf, out=out, workspace=ws)  # noqa: E731
+    dense_on = lambda: atf.prefill(q, k, v, base, kwin, out=out, workspace=ws)  # noqa: E731
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    ms = timed(sparse_on, args.steps)
+    clocks = sampler.stop()
+    ms_off = timed(sparse_off, args.steps)
+    ms_dense = timed(dense_on, args.steps)
+    if atf.device_status() != 0:
+        raise RuntimeError("a kernel's bounded wait ran out in the timed region")
+    per_t = tile_retained_flops(atf, wl, T)
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    vis = (mask_np != 0) | (i == j)[None, None]
+    vis &= (j <= i)[None, None]
+    dist = np.broadcast_to(i - j, vis.shape)
+    flops = float(np.sum(per_t[dist[vis]])) * (Hq // Hkv)
+    density = float(vis.sum()) / (B * Hkv * T * (T + 1) / 2)
+    peaks, src = measured_peaks()
+    long_region = ms * args.steps > 2000.0
+    peak = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
+    achieved = flops / (ms / 1e3) / 1e12
+    line = {"metric": METRIC, "value": round(world * B * N / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(wl, tiles_kept=round(density, 4),
+                           l2="flushed before every step (256 MiB write, outside the timed events)"),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "kernel": f"whole call: rope_pack(q), rope_pack(k), prefill_tc_kernel<{D}, block mask>",
+                         "peak_source": f"{src} ({'sustained' if long_region else 'burst'} bf16)",
+                         "flops_per_launch": flops},
+            "window_off": {"ms_per_step": round(ms_off, 4)},
+            "on_off_speedup": round(ms_off / ms, 4),
+            "dense_window_on": {"ms_per_step": round(ms_dense, 4), "selection_speedup": round(ms_dense / ms, 4)},
+            "gpu_launches": 3 * args.steps, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # Ragged-batch prefill workloads: one step = one varlen prefill call (RoPE pre-pass of
 # the packed Q and K, then the windowed prefill) over sequences of mixed lengths.
 VARLEN_WORKLOADS = {
@@ -159,7 +289,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--workload", default="qwen05b_32k",
-                   choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(VARLEN_WORKLOADS))
+                   choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(VARLEN_WORKLOADS) +
+                   sorted(SPARSE_WORKLOADS))
     p.add_argument("--N", type=int, default=None, help="override sequence length (sweeps)")
     p.add_argument("--k-window", type=float, default=None, help="override k (inf = window off)")
     return p.parse_args()
@@ -839,6 +970,9 @@ def main():
         return
     if args.workload in VARLEN_WORKLOADS:
         run_varlen(args, dict(VARLEN_WORKLOADS[args.workload]))
+        return
+    if args.workload in SPARSE_WORKLOADS:
+        run_sparse(args, dict(SPARSE_WORKLOADS[args.workload]))
         return
     wl = dict(WORKLOADS[args.workload])
     if args.N:

@@ -133,6 +133,28 @@ int atflash_prefill_ex(const void *q, const void *k, const void *v, void *out, i
                        cudaStream_t stream);
 
 /*
+ * Windowed prefill on top of a token-level block selection ("Abstract": token-
+ * level selection such as MInference's is orthogonal to the frequency-level
+ * window, which can be applied on top of it).
+ *   block_mask  DEVICE uint8 [B][Hkv][T][T], T = ceil(N / 128), read during the
+ *               call (stream order), owned by the caller.  Entry (b, g, i, j) != 0
+ *               makes key tile j (keys 128j .. 128j+127) visible to query tile i
+ *               (queries 128i .. 128i+127) for every query head of KV head g.
+ *               The diagonal tile j == i is always visible (each query keeps the
+ *               causal prefix of its own tile, so no row is empty); entries with
+ *               j > i cover only future keys and are ignored.
+ * Query n attends key m iff m <= n and m is visible; the window prunes pair
+ * terms of the visible cells exactly as atflash_prefill_ex, and invisible keys
+ * take no part in the softmax.  q, k, v bf16 (the tensor-core path, D in
+ * {64, 128}); out, out_dtype, lse, workspace and errors as atflash_prefill_ex
+ * (block_mask NULL: ATFLASH_ERR_INVALID_ARG).
+ */
+int atflash_prefill_sparse(const void *q, const void *k, const void *v, const uint8_t *block_mask, void *out,
+                           int B, int Hq, int Hkv, int64_t N, int D, double rope_base, double k_window,
+                           int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/*
  * RoPE pre-pass on its own: rotate x [B][N][H][D] (positions 0..N-1) once and
  * write the layout atflash_prefill_packed reads.
  *   in_dtype ATFLASH_BF16: y is [B*H][D/16][N][16] bf16 ("packed"): chunk c

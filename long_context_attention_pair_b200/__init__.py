@@ -18,7 +18,7 @@ import os
 __all__ = [
     "lib", "prefill", "decode", "pruned_terms", "window_table", "prefill_workspace_bytes",
     "decode_workspace_bytes", "device_status", "AtflashError", "F32", "BF16", "rope_pack", "prefill_packed",
-    "prefill_bf16", "theta_table",
+    "prefill_bf16", "theta_table", "prefill_sparse",
 ]
 
 F32 = 0
@@ -86,12 +86,13 @@ def lib():
         L.atflash_decode_paged_theta.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, dp, d, i, i, i, vp, sz,
                                                  vp]
         L.atflash_prefill_packed_theta.argtypes = [vp, vp, vp, vp, i, i, i, i64, i, dp, d, i, i, vp, vp]
+        L.atflash_prefill_sparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i64, i, d, d, i, vp, vp, sz, vp]
         for f in ("atflash_window_table", "atflash_pruned_terms", "atflash_prefill", "atflash_prefill_ex",
                   "atflash_decode", "atflash_device_status", "atflash_rope_pack", "atflash_prefill_packed",
                   "atflash_prefill_varlen", "atflash_decode_paged", "atflash_theta_table",
                   "atflash_window_table_theta", "atflash_pruned_terms_theta", "atflash_rope_pack_theta",
                   "atflash_prefill_theta", "atflash_decode_theta", "atflash_prefill_varlen_theta",
-                  "atflash_decode_paged_theta", "atflash_prefill_packed_theta"):
+                  "atflash_decode_paged_theta", "atflash_prefill_packed_theta", "atflash_prefill_sparse"):
             getattr(L, f).restype = i
         _lib = L
     return _lib
@@ -211,6 +212,41 @@ def prefill(q, k, v, rope_base: float, k_window: float = math.inf, *, out=None, 
             in_dtype, _dtype_code(out), _dev(lse, "lse") if lse is not None else None, _dev(workspace, "workspace"),
             need, _stream_ptr(stream))
     _check(st, name)
+    return (out, lse) if return_lse else out
+
+
+def prefill_sparse(q, k, v, block_mask, rope_base: float, k_window: float = math.inf, *, out=None, out_dtype=None,
+                   return_lse: bool = False, workspace=None, stream=None):
+    """Windowed prefill on top of a token-level block selection.
+
+    q [B, N, Hq, D], k/v [B, N, Hkv, D] bf16 (un-rotated q/k); block_mask
+    [B, Hkv, T, T] uint8 or bool on the device, T = ceil(N / 128): entry
+    (b, g, i, j) keeps key tile j for query tile i of KV head g's query heads
+    (the diagonal tile always; entries above it are ignored).  Returns out
+    [B, N, Hq, D] and, with ``return_lse``, lse [B, Hq, N] fp32.
+    """
+    torch = _torch()
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    T = (N + 127) // 128
+    if tuple(block_mask.shape) != (B, Hkv, T, T):
+        raise ValueError(f"block_mask must be [{B}, {Hkv}, {T}, {T}], got {tuple(block_mask.shape)}")
+    if block_mask.dtype == torch.bool:
+        block_mask = block_mask.view(torch.uint8)
+    if block_mask.dtype != torch.uint8:
+        raise TypeError("block_mask must be uint8 or bool")
+    if out is None:
+        od = out_dtype if out_dtype is not None else q.dtype
+        out = torch.empty((B, N, Hq, D), dtype=od, device=q.device)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if return_lse else None
+    need = prefill_workspace_bytes(B, Hq, Hkv, N, D, BF16)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib().atflash_prefill_sparse(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(block_mask, "block_mask"),
+                                      _dev(out, "out"), B, Hq, Hkv, N, D, float(rope_base), float(k_window),
+                                      _dtype_code(out), _dev(lse, "lse") if lse is not None else None,
+                                      _dev(workspace, "workspace"), need, _stream_ptr(stream))
+    _check(st, "atflash_prefill_sparse")
     return (out, lse) if return_lse else out
 
 

@@ -191,7 +191,7 @@ static int check_prefill_common(int B, int Hq, int Hkv, int64_t N, int D, const 
 
 static int run_prefill_packed(const void *qt, const void *kt, const void *v, void *out, int B, int Hq, int Hkv,
                               int64_t N, int D, const double *theta, double k, int in_dtype, int out_dtype,
-                              float *lse, cudaStream_t stream) {
+                              float *lse, cudaStream_t stream, const uint8_t *block_mask = nullptr) {
     WindowParams wp;
     int rc = fill_window_theta(wp, D, theta, k, N);
     if (rc != ATFLASH_OK) return rc;
@@ -201,7 +201,8 @@ static int run_prefill_packed(const void *qt, const void *kt, const void *v, voi
     if (in_dtype == ATFLASH_BF16) {
         int *status = device_status_word();
         if (!status) return ATFLASH_ERR_CUDA;
-        e = launch_prefill_tc(qt, kt, v, out, out_f32, lse, p, wp, status, wait_limit_ns(), stream);
+        e = launch_prefill_tc(qt, kt, v, out, out_f32, lse, p, wp, status, wait_limit_ns(), stream, nullptr, 0,
+                              block_mask);
     } else {
         e = launch_prefill_simt_f32((const float *)qt, (const float *)kt, (const float *)v, out, out_f32, lse, p,
                                     wp, stream);
@@ -307,6 +308,28 @@ static int prefill_ex_impl(const void *q, const void *k, const void *v, void *ou
     if ((rc = run_rope_pack(q, qt, B, N, Hq, D, theta, in_dtype, stream)) != ATFLASH_OK) return rc;
     if ((rc = run_rope_pack(k, kt, B, N, Hkv, D, theta, in_dtype, stream)) != ATFLASH_OK) return rc;
     return run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, theta, k_window, in_dtype, out_dtype, lse, stream);
+}
+
+int atflash_prefill_sparse(const void *q, const void *k, const void *v, const uint8_t *block_mask, void *out,
+                           int B, int Hq, int Hkv, int64_t N, int D, double rope_base, double k_window,
+                           int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+    if (!q || !k || !v || !out || !block_mask) return ATFLASH_ERR_INVALID_ARG;
+    BaseTheta bt(D, rope_base);
+    if (bt.rc != ATFLASH_OK) return bt.rc;
+    int rc = check_prefill_common(B, Hq, Hkv, N, D, bt.theta, k_window, ATFLASH_BF16, out_dtype);
+    if (rc != ATFLASH_OK) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATFLASH_ERR_ALIGNMENT;
+    const size_t need = prefill_ws(B, Hq, Hkv, N, D, ATFLASH_BF16);
+    if (!workspace || workspace_bytes < need) return ATFLASH_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATFLASH_ERR_ALIGNMENT;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *qt = ws;
+    void *kt = ws + align256((size_t)B * Hq * N * D * 2);
+    if ((rc = run_rope_pack(q, qt, B, N, Hq, D, bt.theta, ATFLASH_BF16, stream)) != ATFLASH_OK) return rc;
+    if ((rc = run_rope_pack(k, kt, B, N, Hkv, D, bt.theta, ATFLASH_BF16, stream)) != ATFLASH_OK) return rc;
+    return run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, bt.theta, k_window, ATFLASH_BF16, out_dtype, lse,
+                              stream, block_mask);
 }
 
 int atflash_prefill_ex(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,

@@ -50,11 +50,12 @@ cudaError_t launch_prefill_simt_f32(const float *qt, const float *kt, const floa
 // tcgen05 prefill over the packed bf16 Q~/K~ and the caller's bf16 V.
 // cu_seqlens (device, B + 1 entries) != nullptr: q/k/v/out and the packed
 // Q~/K~ hold a batch of `total` tokens packed along the token axis; p.N is the
-// longest sequence.
+// longest sequence.  block_mask (device, [B][Hkv][T][T] uint8, T = ceil(N/128))
+// != nullptr: token-level block selection (not with cu_seqlens).
 cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *v, void *out, int out_f32,
                               float *lse, const Problem &p, const WindowParams &wp, int *status,
                               uint64_t wait_limit_ns, cudaStream_t s, const int32_t *cu_seqlens = nullptr,
-                              int64_t total = 0);
+                              int64_t total = 0, const uint8_t *block_mask = nullptr);
 
 // Split-KV decode + merge.
 int decode_split_keys(int B, int Hkv, int64_t Nmax);

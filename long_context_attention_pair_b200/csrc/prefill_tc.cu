@@ -164,6 +164,24 @@ struct BandWalk {
     }
 };
 
+// The key tiles a CTA visits, in order: all of 0..qt, or under a token-level
+// block selection the tiles whose mask entry is set, the diagonal tile qt always
+// (every query keeps at least the causal prefix of its own tile).  Every warp
+// walks the same sequence; pipeline stages and phases count visited tiles.
+template <bool kMasked>
+struct KeyTiles {
+    const uint8_t *row;  // mask entries of this CTA's (sequence, KV head, query tile)
+    int qt;
+    __device__ __forceinline__ int from(int j) const {
+        if constexpr (kMasked) {
+            while (j < qt && row[j] == 0) ++j;
+        }
+        return j;
+    }
+    __device__ __forceinline__ int first() const { return from(0); }
+    __device__ __forceinline__ int after(int j) const { return from(j + 1); }
+};
+
 __device__ __forceinline__ bool wait_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
@@ -175,12 +193,14 @@ __device__ __forceinline__ bool wait_drain(uint64_t *bar, uint32_t parity, uint6
 // kVarlen: the batch is packed along the token axis (q, k, v, out [total][H][D],
 // packed Q~/K~ [H][D/16][total][16]); sequence b holds tokens cu[b]..cu[b+1]-1
 // and N is the longest sequence.  Otherwise q/k/v/out are [B][N][H][D].
-template <int D, bool kVarlen, int NH>
+// kMasked: token-level block selection, block_mask [B][Hkv][T][T] (T query /
+// key tiles of 128), entry (b, g, i, j) != 0 keeps key tile j for query tile i.
+template <int D, bool kVarlen, int NH, bool kMasked>
 __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ WindowParams wp,
                       void *out, int out_f32, float *lse, int64_t N, int Hq, int Hkv, int *status,
-                      uint64_t limit_ns, const int32_t *cu_seqlens, int64_t total) {
+                      uint64_t limit_ns, const int32_t *cu_seqlens, int64_t total, const uint8_t *block_mask) {
     using F = Cfg<D, NH>;
     using W = Warps<NH>;
     constexpr int kThreads = W::Threads;
@@ -211,6 +231,9 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
     const int nwg = two ? 2 : 1;
     const int64_t n0 = (int64_t)qt * kBM;
     const int nkt = qt + 1;  // key tiles 0..qt (causal)
+    KeyTiles<kMasked> tiles;
+    tiles.qt = qt;
+    tiles.row = kMasked ? block_mask + (((size_t)b * Hkv + kvh) * num_qt + qt) * (size_t)num_qt : nullptr;
     // Where this CTA's sequence lives: first token on the token axis, valid rows,
     // batch coordinate of the tensor maps, rows per batch of out / lse.
     int64_t tokbase = 0, seq_len = N, nrows = N;
@@ -288,24 +311,24 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
             bool ok = true;
             BandWalk bw;
             bw.init(w, H, n0);
-            for (int j = 0; j < nkt && ok; ++j) {
-                const int ks = j % KS, vs = j % VS;
+            for (int it = 0, j = tiles.first(); j < nkt && ok; ++it, j = tiles.after(j)) {
+                const int ks = it % KS, vs = it % VS;
                 const int64_t m0 = (int64_t)j * kBN;
                 const int ca = bw.at(w, n0, m0).r_lo >> 3;
                 wc.site = 1;
-                if (!(ok = mbar_wait(&ctl->k_empty[ks], ((j / KS) & 1) ^ 1, wc))) break;
+                if (!(ok = mbar_wait(&ctl->k_empty[ks], ((it / KS) & 1) ^ 1, wc))) break;
                 mbar_expect_tx(&ctl->k_full[ks], (uint32_t)(C - ca) * kChunkBytes);
                 for (int c = ca; c < C; ++c)
                     tma_load_3d(sK + ks * F::KBytes + c * kChunkBytes, &tm_k, &ctl->k_full[ks], 0,
                                 (int)(tokbase + m0), (bz * Hkv + kvh) * C + c);
-                last_k[ks] = j;
+                last_k[ks] = it;
                 wc.site = 2;
-                if (!(ok = mbar_wait(&ctl->v_empty[vs], ((j / VS) & 1) ^ 1, wc))) break;
+                if (!(ok = mbar_wait(&ctl->v_empty[vs], ((it / VS) & 1) ^ 1, wc))) break;
                 mbar_expect_tx(&ctl->v_full[vs], F::VBytes);
                 for (int gidx = 0; gidx < D / 64; ++gidx)
                     tma_load_4d(sV + vs * F::VBytes + gidx * 16384, &tm_v, &ctl->v_full[vs], gidx * 64, kvh,
                                 (int)(tokbase + m0), bz);
-                last_v[vs] = j;
+                last_v[vs] = it;
             }
             if (!ok) {
                 // Let every copy this thread started land before the CTA exits.
@@ -322,13 +345,13 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
         bool ok = true;
         BandWalk bw;
         bw.init(w, H, n0);
-        for (int j = 0; j < nkt && ok; ++j) {
-            const int ks = j % KS;
+        for (int it = 0, j = tiles.first(); j < nkt && ok; ++it, j = tiles.after(j)) {
+            const int ks = it % KS;
             const Band bd = bw.at(w, n0, (int64_t)j * kBN);
             const int r_lo = bd.r_lo;
             const int ca = r_lo >> 3;
             wc.site = 3;
-            if (!(ok = mbar_wait_warp(&ctl->k_full[ks], (j / KS) & 1, wc))) break;
+            if (!(ok = mbar_wait_warp(&ctl->k_full[ks], (it / KS) & 1, wc))) break;
             // Boundary pairs r_lo + b: key values of keys (2i, 2i+1) as
             // (k_r[2i], k_r[2i+1], k_{r+H}[2i], k_{r+H}[2i+1]) in fp32.
             const int nb = min(bd.r_full - r_lo, kMaxStagedPairs);
@@ -377,24 +400,24 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
         };
         BandWalk bw;
         bw.init(w, H, n0);
-        for (int j = 0; j < nkt && ok; ++j) {
-            const int ks = j % KS;
+        for (int it = 0, j = tiles.first(); j < nkt && ok; ++it, j = tiles.after(j)) {
+            const int ks = it % KS;
             const int ca = bw.at(w, n0, (int64_t)j * kBN).r_lo >> 3;
             wc.site = 7;
-            if (!(ok = mbar_wait_warp(&ctl->k_ready[ks], (j / KS) & 1, wc))) break;
+            if (!(ok = mbar_wait_warp(&ctl->k_ready[ks], (it / KS) & 1, wc))) break;
             // S_0(j) once its columns are free: read by head 0 (own buffer) or by
             // head 1 (buffer shared by the two heads); S_1(j) likewise.
             wc.site = 13;
-            if (j > 0) {
+            if (it > 0) {
                 uint64_t *free_bar = (F::SharedS && two) ? &ctl->s_read[1] : &ctl->s_read[0];
-                if (!(ok = mbar_wait_warp(free_bar, (j - 1) & 1, wc))) break;
+                if (!(ok = mbar_wait_warp(free_bar, (it - 1) & 1, wc))) break;
             }
             issue_qk(0, ks, ca);
             if (two) {
                 if (F::SharedS) {
-                    if (!(ok = mbar_wait_warp(&ctl->s_read[0], j & 1, wc))) break;
-                } else if (j > 0) {
-                    if (!(ok = mbar_wait_warp(&ctl->s_read[1], (j - 1) & 1, wc))) break;
+                    if (!(ok = mbar_wait_warp(&ctl->s_read[0], it & 1, wc))) break;
+                } else if (it > 0) {
+                    if (!(ok = mbar_wait_warp(&ctl->s_read[1], (it - 1) & 1, wc))) break;
                 }
                 issue_qk(1, ks, ca);
             }
@@ -406,13 +429,13 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
         const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
         const uint32_t sVa = smem_u32(sV);
         bool ok = true;
-        for (int j = 0; j < nkt && ok; ++j) {
-            const int vs = j % VS;
+        for (int it = 0, j = tiles.first(); j < nkt && ok; ++it, j = tiles.after(j)) {
+            const int vs = it % VS;
             wc.site = 5;
-            if (!(ok = mbar_wait_warp(&ctl->v_full[vs], (j / VS) & 1, wc))) break;
+            if (!(ok = mbar_wait_warp(&ctl->v_full[vs], (it / VS) & 1, wc))) break;
             for (int t = 0; t < nwg && ok; ++t) {
                 wc.site = 6;
-                if (!(ok = mbar_wait_warp(&ctl->p_full[t], j & 1, wc))) break;
+                if (!(ok = mbar_wait_warp(&ctl->p_full[t], it & 1, wc))) break;
                 if (lane == 0) {
                     tc_fence_after();
                     const uint32_t o_col = t ? F::TmemO1 : F::TmemO0;
@@ -422,7 +445,7 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                         // B = V rows [16kk, 16kk+16): MN-major SW128, 64-dim groups 16 KB apart.
                         const uint64_t db = smem_desc(sVa + vs * F::VBytes + kk * 2048, 16384, 1024, kSwizzle128B);
                         umma_bf16_ts(tmem + o_col, tmem + (t ? F::TmemP1 : F::TmemP0) + kk * 8, db, idesc_pv,
-                                     (j > 0 || kk > 0) ? 1u : 0u);
+                                     (it > 0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(&ctl->o_done[t]);
                 }
@@ -451,13 +474,14 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
             bool ok = mbar_wait_warp(&ctl->q_full, 0, wc);  // Q~ rows are read for the boundary fix-up
             BandWalk bw;
             bw.init(w, H, n0);
-            for (int j = 0; j < nkt && ok; ++j) {
-                const int ks = j % KS;
+            int it = 0;  // key tiles visited
+            for (int j = tiles.first(); j < nkt && ok; ++it, j = tiles.after(j)) {
+                const int ks = it % KS;
                 const int64_t m0 = (int64_t)j * kBN;
                 const Band bd = bw.at(w, n0, m0);
                 float s[kBN];
                 wc.site = 9;
-                if (!(ok = mbar_wait_warp(&ctl->s_full[t], j & 1, wc))) break;
+                if (!(ok = mbar_wait_warp(&ctl->s_full[t], it & 1, wc))) break;
                 tc_fence_after();
                 if ((bd.r_lo >> 3) < C) {
                     uint32_t r0[32], r1[32], r2[32], r3[32];
@@ -492,7 +516,7 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                     // S(j) was waited for above and its MMA waited for this phase, and
                     // the stage's next phase needs this warp to release the stage first.
                     wc.site = 10;
-                    if (!(ok = mbar_wait_warp(&ctl->k_ready[ks], (j / KS) & 1, wc))) break;
+                    if (!(ok = mbar_wait_warp(&ctl->k_ready[ks], (it / KS) & 1, wc))) break;
                     const float4 *bst = sBnd + ks * (kMaxStagedPairs * 64);
                     for (int r = bd.r_lo; r < bd.r_full; ++r) {
                         const int lim = (int)(n - m0 - (int64_t)w[r]);
@@ -573,8 +597,8 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                 // other loads S, corrects it and stores P.
                 if (F::Token && two) {
                     wc.site = 14;
-                    if (t == 1) ok = mbar_wait_warp(&ctl->tok[0][q4], j & 1, wc);
-                    else if (j > 0) ok = mbar_wait_warp(&ctl->tok[1][q4], (j - 1) & 1, wc);
+                    if (t == 1) ok = mbar_wait_warp(&ctl->tok[0][q4], it & 1, wc);
+                    else if (it > 0) ok = mbar_wait_warp(&ctl->tok[1][q4], (it - 1) & 1, wc);
                     if (!ok) break;
                 }
                 // P = exp2(s * scale - m) as bf16 pairs; S registers die as P is produced.
@@ -609,10 +633,10 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                 }
                 // Rescale O only when some row's max grew past the threshold (rare).
                 // PV_t(j-1) must also be done reading P_t before it is overwritten.
-                const bool rescale = (j > 0) && __any_sync(0xffffffffu, need);
-                if (j > 0) {
+                const bool rescale = (it > 0) && __any_sync(0xffffffffu, need);
+                if (it > 0) {
                     wc.site = 11;
-                    if (!(ok = mbar_wait_warp(&ctl->o_done[t], (j - 1) & 1, wc))) break;
+                    if (!(ok = mbar_wait_warp(&ctl->o_done[t], (it - 1) & 1, wc))) break;
                     tc_fence_after();
                 }
                 if (rescale) {
@@ -642,7 +666,7 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
             }
             if (ok) {
                 wc.site = 12;
-                ok = mbar_wait_warp(&ctl->o_done[t], (nkt - 1) & 1, wc);
+                ok = mbar_wait_warp(&ctl->o_done[t], (it - 1) & 1, wc);
             }
             if (ok) {
                 tc_fence_after();
@@ -714,9 +738,12 @@ static cudaError_t make_map(CUtensorMap *map, void *base, int rank, const cuuint
 
 cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *v, void *out, int out_f32,
                               float *lse, const Problem &p, const WindowParams &wp, int *status,
-                              uint64_t wait_limit_ns, cudaStream_t s, const int32_t *cu_seqlens, int64_t total) {
+                              uint64_t wait_limit_ns, cudaStream_t s, const int32_t *cu_seqlens, int64_t total,
+                              const uint8_t *block_mask) {
     const int C = p.D / 16;
     const bool varlen = cu_seqlens != nullptr;
+    const bool masked = block_mask != nullptr;
+    if (varlen && masked) return cudaErrorInvalidValue;
     // Token axis of the maps: N per batch entry, or the whole packed batch.
     const cuuint64_t T = varlen ? (cuuint64_t)total : (cuuint64_t)p.N;
     const cuuint64_t NB = varlen ? 1 : (cuuint64_t)p.B;
@@ -745,15 +772,28 @@ cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *
     const int num_qt = (int)((p.N + tc::kBM - 1) / tc::kBM);
     const int G = p.Hq / p.Hkv;
     cudaError_t e;
-#define ATF_PREFILL_TC(DD, VL, NHH)                                                                              \
+#define ATF_PREFILL_TC_M(DD, VL, NHH, MK)                                                                        \
     do {                                                                                                         \
         const int smem = tc::Cfg<DD, NHH>::Request;                                                             \
         dim3 grid((unsigned)num_qt, (unsigned)(p.B * p.Hkv * ((G + NHH - 1) / NHH)));                          \
-        e = cudaFuncSetAttribute(tc::prefill_tc_kernel<DD, VL, NHH>,                                            \
+        e = cudaFuncSetAttribute(tc::prefill_tc_kernel<DD, VL, NHH, MK>,                                        \
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                             \
         if (e != cudaSuccess) return e;                                                                          \
-        tc::prefill_tc_kernel<DD, VL, NHH><<<grid, tc::Warps<NHH>::Threads, smem, s>>>(                         \
-            tq, tk, tv, wp, out, out_f32, lse, p.N, p.Hq, p.Hkv, status, wait_limit_ns, cu_seqlens, total);      \
+        tc::prefill_tc_kernel<DD, VL, NHH, MK><<<grid, tc::Warps<NHH>::Threads, smem, s>>>(                     \
+            tq, tk, tv, wp, out, out_f32, lse, p.N, p.Hq, p.Hkv, status, wait_limit_ns, cu_seqlens, total,       \
+            block_mask);                                                                                         \
+    } while (0)
+    // Block-selected launches (never varlen) take their own instantiations, so that
+    // the dense kernels' code is what it was.
+#define ATF_PREFILL_TC(DD, VL, NHH)                                                                              \
+    do {                                                                                                         \
+        if constexpr (!VL) {                                                                                     \
+            if (masked) {                                                                                        \
+                ATF_PREFILL_TC_M(DD, false, NHH, true);                                                          \
+                break;                                                                                           \
+            }                                                                                                    \
+        }                                                                                                        \
+        ATF_PREFILL_TC_M(DD, VL, NHH, false);                                                                    \
     } while (0)
     if (p.D == 128) {
         if (varlen) ATF_PREFILL_TC(128, true, 2); else ATF_PREFILL_TC(128, false, 2);
@@ -772,6 +812,7 @@ cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *
         return cudaErrorInvalidValue;
     }
 #undef ATF_PREFILL_TC
+#undef ATF_PREFILL_TC_M
     return cudaGetLastError();
 }
 

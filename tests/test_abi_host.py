@@ -117,6 +117,29 @@ def test_prefill_argument_errors(L):
     assert prefill_ex(L, ws=ctypes.c_void_p((1 << 20) + 16)) == -6
 
 
+def prefill_sparse(L, **kw):
+    a = dict(q=P, k=P, v=P, mask=P, out=P, B=1, Hq=2, Hkv=1, N=256, D=64, base=1e4, kwin=1.0, outd=atf.BF16,
+             lse=None, ws=P, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return L.atflash_prefill_sparse(a["q"], a["k"], a["v"], a["mask"], a["out"], a["B"], a["Hq"], a["Hkv"], a["N"],
+                                    a["D"], a["base"], a["kwin"], a["outd"], a["lse"], a["ws"], a["wsb"],
+                                    a["stream"])
+
+
+def test_prefill_sparse_argument_errors(L):
+    assert prefill_sparse(L, mask=None) == -1
+    assert prefill_sparse(L, q=None) == -1
+    assert prefill_sparse(L, Hq=3, Hkv=2) == -1
+    assert prefill_sparse(L, kwin=float("nan")) == -1
+    assert prefill_sparse(L, base=0.5) == -1
+    assert prefill_sparse(L, D=96) == -2       # bf16 tensor-core path only
+    assert prefill_sparse(L, outd=9) == -2
+    assert prefill_sparse(L, out=ctypes.c_void_p((1 << 20) + 8)) == -6
+    assert prefill_sparse(L, ws=None) == -3
+    assert prefill_sparse(L, wsb=100) == -3
+    assert prefill_sparse(L, ws=ctypes.c_void_p((1 << 20) + 16)) == -6
+
+
 def test_rope_pack_and_packed_prefill_argument_errors(L):
     assert L.atflash_rope_pack(None, P, 1, 256, 2, 64, 1e4, atf.BF16, None) == -1
     assert L.atflash_rope_pack(P, P, 1, 256, 2, 96, 1e4, atf.BF16, None) == -2

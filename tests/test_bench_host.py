@@ -59,3 +59,27 @@ def test_captured_traffic_is_reported_only_for_its_own_workload():
     assert bench.prefill_traffic("qwen05b_32k", dict(wl, N=65536)) is None
     assert bench.prefill_traffic("qwen05b_32k", dict(wl, k_window=float("inf"))) is None
     assert bench.decode_traffic("decode_128k", 1 << 17) is None
+
+
+def test_tile_flops_sum_to_the_dense_retained_flops():
+    # Summed over every causal tile pair, the per-distance tile FLOPs of the
+    # block-selected lines equal the closed-form retained FLOPs of one head.
+    import long_context_attention_pair_b200 as atf
+    for wl in bench.SPARSE_WORKLOADS.values():
+        T = wl["N"] // 128
+        per_t = bench.tile_retained_flops(atf, wl, T)
+        terms = atf.pruned_terms(wl["N"], wl["D"], wl["rope_base"], wl["k_window"])
+        dense = 4 * terms["kept"] + wl["D"] * wl["N"] * (wl["N"] + 1)
+        assert sum(per_t[t] * (T - t) for t in range(T)) == dense
+
+
+def test_block_mask_recipe_shape_and_structure():
+    import numpy as np
+    wl = bench.SPARSE_WORKLOADS["qwen05b_32k_sparse"]
+    T = wl["N"] // 128
+    m = bench.block_mask_recipe(wl, T)
+    assert m.shape == (wl["B"], wl["Hkv"], T, T) and m.dtype == np.uint8
+    assert not np.any(np.triu(m[0, 0], 1))                      # causal tiles only
+    assert np.all(np.diag(m[0, 0]) == 1)                         # local band includes the diagonal
+    assert np.all(m[0, :, wl["sink_tiles"]:, :wl["sink_tiles"]] == 1)
+    assert np.array_equal(m, bench.block_mask_recipe(wl, T))    # seeded
