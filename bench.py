@@ -268,8 +268,8 @@ KERNELS_PER_STEP = 5  # rope_pack(q), rope_pack(k), prefill_tc, decode_split, de
 # DRAM bytes per launch of the tcgen05 prefill kernel on this workload, from one
 # ncu capture (profiles/prefill_tc_qwen05b_32k.md).  Valid only while the
 # kernel source hashes to `source_sha1`; otherwise the line reports null.
-TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98524672,
-           "source_sha1": "1f685c21a7d0dcaf521156fdca2c5f034adce7b8"}
+TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98168320,
+           "source_sha1": "fd039e524fa9ed078dfba5e3b08f3de1cb0a5392"}
 # DRAM bytes per launch of the decode kernel (split states included, merge not) on
 # the full-size workloads, from single-pass ncu captures
 # (profiles/decode_tc_qwen7b_packed_4x128k.md); valid while decode_tc.cu hashes to

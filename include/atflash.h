@@ -278,6 +278,10 @@ int atflash_rope_pack_theta(const void *x, void *y, int B, int64_t N, int H, int
 int atflash_prefill_theta(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
                           int64_t N, int D, const double *theta, double k_window, int in_dtype, int out_dtype,
                           float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+int atflash_prefill_sparse_theta(const void *q, const void *k, const void *v, const uint8_t *block_mask,
+                                 void *out, int B, int Hq, int Hkv, int64_t N, int D, const double *theta,
+                                 double k_window, int out_dtype, float *lse, void *workspace,
+                                 size_t workspace_bytes, cudaStream_t stream);
 /* qpack/kpack written by atflash_rope_pack_theta with the same table. */
 int atflash_prefill_packed_theta(const void *qpack, const void *kpack, const void *v, void *out, int B, int Hq,
                                  int Hkv, int64_t N, int D, const double *theta, double k_window, int in_dtype,

@@ -87,12 +87,14 @@ def lib():
                                                  vp]
         L.atflash_prefill_packed_theta.argtypes = [vp, vp, vp, vp, i, i, i, i64, i, dp, d, i, i, vp, vp]
         L.atflash_prefill_sparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i64, i, d, d, i, vp, vp, sz, vp]
+        L.atflash_prefill_sparse_theta.argtypes = [vp, vp, vp, vp, vp, i, i, i, i64, i, dp, d, i, vp, vp, sz, vp]
         for f in ("atflash_window_table", "atflash_pruned_terms", "atflash_prefill", "atflash_prefill_ex",
                   "atflash_decode", "atflash_device_status", "atflash_rope_pack", "atflash_prefill_packed",
                   "atflash_prefill_varlen", "atflash_decode_paged", "atflash_theta_table",
                   "atflash_window_table_theta", "atflash_pruned_terms_theta", "atflash_rope_pack_theta",
                   "atflash_prefill_theta", "atflash_decode_theta", "atflash_prefill_varlen_theta",
-                  "atflash_decode_paged_theta", "atflash_prefill_packed_theta", "atflash_prefill_sparse"):
+                  "atflash_decode_paged_theta", "atflash_prefill_packed_theta", "atflash_prefill_sparse",
+                  "atflash_prefill_sparse_theta"):
             getattr(L, f).restype = i
         _lib = L
     return _lib
@@ -216,7 +218,7 @@ def prefill(q, k, v, rope_base: float, k_window: float = math.inf, *, out=None, 
 
 
 def prefill_sparse(q, k, v, block_mask, rope_base: float, k_window: float = math.inf, *, out=None, out_dtype=None,
-                   return_lse: bool = False, workspace=None, stream=None):
+                   return_lse: bool = False, workspace=None, stream=None, theta=None):
     """Windowed prefill on top of a token-level block selection.
 
     q [B, N, Hq, D], k/v [B, N, Hkv, D] bf16 (un-rotated q/k); block_mask
@@ -242,11 +244,13 @@ def prefill_sparse(q, k, v, block_mask, rope_base: float, k_window: float = math
     need = prefill_workspace_bytes(B, Hq, Hkv, N, D, BF16)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    st = lib().atflash_prefill_sparse(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(block_mask, "block_mask"),
-                                      _dev(out, "out"), B, Hq, Hkv, N, D, float(rope_base), float(k_window),
-                                      _dtype_code(out), _dev(lse, "lse") if lse is not None else None,
-                                      _dev(workspace, "workspace"), need, _stream_ptr(stream))
-    _check(st, "atflash_prefill_sparse")
+    fn, name, rope = lib().atflash_prefill_sparse, "atflash_prefill_sparse", float(rope_base)
+    if theta is not None:
+        fn, name, rope = lib().atflash_prefill_sparse_theta, "atflash_prefill_sparse_theta", _theta_arg(theta, D)
+    st = fn(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(block_mask, "block_mask"), _dev(out, "out"), B, Hq, Hkv,
+            N, D, rope, float(k_window), _dtype_code(out), _dev(lse, "lse") if lse is not None else None,
+            _dev(workspace, "workspace"), need, _stream_ptr(stream))
+    _check(st, name)
     return (out, lse) if return_lse else out
 
 

@@ -310,14 +310,11 @@ static int prefill_ex_impl(const void *q, const void *k, const void *v, void *ou
     return run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, theta, k_window, in_dtype, out_dtype, lse, stream);
 }
 
-int atflash_prefill_sparse(const void *q, const void *k, const void *v, const uint8_t *block_mask, void *out,
-                           int B, int Hq, int Hkv, int64_t N, int D, double rope_base, double k_window,
-                           int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
-                           cudaStream_t stream) {
-    if (!q || !k || !v || !out || !block_mask) return ATFLASH_ERR_INVALID_ARG;
-    BaseTheta bt(D, rope_base);
-    if (bt.rc != ATFLASH_OK) return bt.rc;
-    int rc = check_prefill_common(B, Hq, Hkv, N, D, bt.theta, k_window, ATFLASH_BF16, out_dtype);
+static int prefill_sparse_impl(const void *q, const void *k, const void *v, const uint8_t *block_mask, void *out,
+                               int B, int Hq, int Hkv, int64_t N, int D, const double *theta, double k_window,
+                               int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
+    int rc = check_prefill_common(B, Hq, Hkv, N, D, theta, k_window, ATFLASH_BF16, out_dtype);
     if (rc != ATFLASH_OK) return rc;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATFLASH_ERR_ALIGNMENT;
     const size_t need = prefill_ws(B, Hq, Hkv, N, D, ATFLASH_BF16);
@@ -326,10 +323,30 @@ int atflash_prefill_sparse(const void *q, const void *k, const void *v, const ui
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     void *qt = ws;
     void *kt = ws + align256((size_t)B * Hq * N * D * 2);
-    if ((rc = run_rope_pack(q, qt, B, N, Hq, D, bt.theta, ATFLASH_BF16, stream)) != ATFLASH_OK) return rc;
-    if ((rc = run_rope_pack(k, kt, B, N, Hkv, D, bt.theta, ATFLASH_BF16, stream)) != ATFLASH_OK) return rc;
-    return run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, bt.theta, k_window, ATFLASH_BF16, out_dtype, lse,
+    if ((rc = run_rope_pack(q, qt, B, N, Hq, D, theta, ATFLASH_BF16, stream)) != ATFLASH_OK) return rc;
+    if ((rc = run_rope_pack(k, kt, B, N, Hkv, D, theta, ATFLASH_BF16, stream)) != ATFLASH_OK) return rc;
+    return run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, theta, k_window, ATFLASH_BF16, out_dtype, lse,
                               stream, block_mask);
+}
+
+int atflash_prefill_sparse(const void *q, const void *k, const void *v, const uint8_t *block_mask, void *out,
+                           int B, int Hq, int Hkv, int64_t N, int D, double rope_base, double k_window,
+                           int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+    if (!q || !k || !v || !out || !block_mask) return ATFLASH_ERR_INVALID_ARG;
+    BaseTheta bt(D, rope_base);
+    if (bt.rc != ATFLASH_OK) return bt.rc;
+    return prefill_sparse_impl(q, k, v, block_mask, out, B, Hq, Hkv, N, D, bt.theta, k_window, out_dtype, lse,
+                               workspace, workspace_bytes, stream);
+}
+
+int atflash_prefill_sparse_theta(const void *q, const void *k, const void *v, const uint8_t *block_mask,
+                                 void *out, int B, int Hq, int Hkv, int64_t N, int D, const double *theta,
+                                 double k_window, int out_dtype, float *lse, void *workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+    if (!q || !k || !v || !out || !block_mask) return ATFLASH_ERR_INVALID_ARG;
+    return prefill_sparse_impl(q, k, v, block_mask, out, B, Hq, Hkv, N, D, theta, k_window, out_dtype, lse,
+                               workspace, workspace_bytes, stream);
 }
 
 int atflash_prefill_ex(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,

@@ -528,7 +528,6 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                         const float2 qb2 = make_float2(bf16hi(qw), bf16hi(qw));
                         if (r - bd.r_lo < kMaxStagedPairs) {
                             const float4 *kb = bst + (r - bd.r_lo) * 64;
-#pragma unroll
                             // One predicated loop per 32-column block: a separate copy for the
                             // blocks every row of the warp prunes in full measured slower (the
                             // larger correction code cost more than the saved compares).

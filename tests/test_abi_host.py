@@ -295,6 +295,8 @@ def test_theta_tables_rejected(L):
                                             atf.F32, P, 1 << 40, None) == -1, name
         assert L.atflash_prefill_packed_theta(P, P, P, P, 1, 2, 1, 256, 64, arr, 1.0, atf.BF16, atf.BF16, None,
                                               None) == -1, name
+        assert L.atflash_prefill_sparse_theta(P, P, P, P, P, 1, 2, 1, 256, 64, arr, 1.0, atf.BF16, None, P,
+                                              1 << 40, None) == -1, name
     assert L.atflash_prefill_theta(P, P, P, P, 1, 2, 1, 256, 64, None, 1.0, atf.BF16, atf.BF16, None, P,
                                    1 << 40, None) == -1
     assert L.atflash_prefill_packed_theta(P, P, P, P, 1, 2, 1, 256, 64, None, 1.0, atf.BF16, atf.BF16, None,

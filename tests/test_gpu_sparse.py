@@ -141,3 +141,26 @@ def test_sparse_bench_workload_sampled(oracle, name, rows):
     ref = oracle.prefill_rows_sparse(P.host(q[0, idx]), sel, P.host(k[0]), P.host(v[0]), wl["rope_base"],
                                      wl["k_window"], mask[0], 128)
     P.check(P.host(out[0, idx]), ref, "bf16", name)
+
+
+def test_theta_table_variant(oracle):
+    # The base table through the _theta call is bit-identical to the base-taking
+    # call; a scaled table matches the oracle with the same table installed.
+    from scaled import llama3_scaled_theta
+    B, N, Hq, Hkv, D, base, kwin = 1, 1500, 4, 2, 128, 5e5, 16.0
+    T = (N + 127) // 128
+    q = P.gen(99, "q", (B, N, Hq, D), "bf16")
+    k = P.gen(99, "k", (B, N, Hkv, D), "bf16")
+    v = P.gen(99, "v", (B, N, Hkv, D), "bf16")
+    mask = random_mask(B, Hkv, T, 0.4, 100)
+    m = torch.as_tensor(mask, device="cuda")
+    a = atf.prefill_sparse(q, k, v, m, base, kwin)
+    b = atf.prefill_sparse(q, k, v, m, 0.0, kwin, theta=atf.theta_table(D, base))
+    th = llama3_scaled_theta(D, base, factor=32.0, orig_ctx=256.0)
+    c = atf.prefill_sparse(q, k, v, m, 0.0, kwin, theta=th, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    with oracle.scaled_rope(th):
+        ref = oracle.prefill_rows_sparse(P.host(q[0]), np.arange(N), P.host(k[0]), P.host(v[0]), base, kwin, mask[0],
+                                         128)
+    P.check(P.host(c[0]), ref, "bf16", "scaled sparse")
