@@ -10,6 +10,12 @@ per step) with inputs resident in HBM; L2 (126 MB) is flushed before every
 step by writing a 256 MiB buffer outside the timed events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --workload NAME ...
+
+Other workloads (`--workload`): the prefill shapes of the larger models
+(WORKLOADS), decode over contiguous or paged caches (DECODE_WORKLOADS), ragged
+batches (VARLEN_WORKLOADS) and the window over a block selection
+(SPARSE_WORKLOADS); each prints the same kind of line for its own step.
 
 N > 1 (torchrun): every rank runs an independent replica of the workload on
 its own GPU (the path has no exchange step); time = max over ranks.
@@ -181,6 +187,10 @@ def run_sparse(args, wl):
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     B, N, Hq, Hkv, D = wl["B"], wl["N"], wl["Hq"], wl["Hkv"], wl["D"]
     base, kwin = wl["rope_base"], wl["k_window"]
     T = (N + 127) // 128
@@ -213,10 +223,10 @@ def run_sparse(args, wl):
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    ms = timed(sparse_on, args.steps)
+    ms = reduce_max(timed(sparse_on, args.steps), world, dev)
     clocks = sampler.stop()
-    ms_off = timed(sparse_off, args.steps)
-    ms_dense = timed(dense_on, args.steps)
+    ms_off = reduce_max(timed(sparse_off, args.steps), world, dev)
+    ms_dense = reduce_max(timed(dense_on, args.steps), world, dev)
     if atf.device_status() != 0:
         raise RuntimeError("a kernel's bounded wait ran out in the timed region")
     per_t = tile_retained_flops(atf, wl, T)
@@ -247,6 +257,9 @@ def run_sparse(args, wl):
             "gpu_launches": 3 * args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
 
 
 # Ragged-batch prefill workloads: one step = one varlen prefill call (RoPE pre-pass of
@@ -649,6 +662,10 @@ def run_decode(args, wl):
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     B, Hq, Hkv, D, L = wl["B"], wl["Hq"], wl["Hkv"], wl["D"], wl["N"]
     base, kwin = wl["rope_base"], wl["k_window"]
     q = synthetic.tensor_torch(wl["seed"], "q_dec", (B, Hq, D), "bf16", device=dev)
@@ -709,9 +726,9 @@ def run_decode(args, wl):
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    ms = timed(kwin, args.steps)
+    ms = reduce_max(timed(kwin, args.steps), world, dev)
     clocks = sampler.stop()
-    ms_off = timed(math.inf, args.steps)
+    ms_off = reduce_max(timed(math.inf, args.steps), world, dev)
     if atf.device_status() != 0:
         raise RuntimeError("a kernel's bounded wait ran out in the timed region")
     peaks, src = measured_peaks()
@@ -732,6 +749,9 @@ def run_decode(args, wl):
             "on_off_speedup": round(ms_off / ms, 4), "gpu_launches": 2 * args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
 
 
 def ragged_lengths(seed, total, lo, hi):
