@@ -406,3 +406,19 @@ def test_sparse_diagonal_and_future_entries_are_ignored(oracle):
     ref = attention_textbook(q[16:n + 1, 0], k[16:n + 1, 0], v[16:n + 1, 0], base)[-1]
     # the textbook attention above starts positions at 0; RoPE scores depend on n - m only
     np.testing.assert_allclose(only_diag[n, 0], ref, rtol=0, atol=1e-12)
+
+
+def test_sparse_under_scaled_table_all_visible_equals_dense(oracle):
+    # The block-selected rows take the installed frequency table like the dense ones.
+    from scaled import llama3_scaled_theta
+    N, D, Hq, Hkv, tile, base = 80, 32, 2, 1, 16, 1e4
+    T = (N + tile - 1) // tile
+    th = llama3_scaled_theta(D, base, factor=8.0, orig_ctx=64.0)
+    q, k, v = rand((N, Hq, D), 101), rand((N, Hkv, D), 102, "k"), rand((N, Hkv, D), 103, "v")
+    rows = np.arange(N)
+    with oracle.scaled_rope(th):
+        dense = oracle.prefill_rows(q, rows, k, v, base, 1.0)
+        sparse = oracle.prefill_rows_sparse(q, rows, k, v, base, 1.0, np.ones((Hkv, T, T), np.uint8), tile)
+    plain = oracle.prefill_rows(q, rows, k, v, base, 1.0)
+    assert np.array_equal(dense, sparse)
+    assert not np.allclose(dense, plain)
