@@ -1,13 +1,17 @@
 #!/usr/bin/env python
 """Benchmark of the windowed-attention hot path; prints ONE JSON line (rank 0).
 
-Workload (default): Qwen2.5-0.5B-shaped single-layer prefill, B=1, Hq=14,
-Hkv=2 (GQA), D=64, RoPE base 1e6, N=32768, k=8, bf16 inputs i.i.d. N(0,1)
-from seed 1, plus the decode of the last row against the same K/V.  One step =
-RoPE pre-pass (q and k) -> windowed tcgen05 prefill -> split-KV decode ->
-merge: every row of the hot path.  `value` is prefill tokens/s (B*N tokens
-per step) with inputs resident in HBM; L2 (126 MB) is flushed before every
-step by writing a 256 MiB buffer outside the timed events.
+Workload (default): Qwen2.5-7B-1M-shaped single-layer prefill, B=1, Hq=28,
+Hkv=4 (GQA), D=128, RoPE base 1e7, N=524288, k=16, bf16 inputs i.i.d. N(0,1)
+from seed 3, plus the decode of the last row against the same K/V.  One step =
+RoPE pre-pass (q and k) -> windowed tcgen05 prefill -> fp32 short rows ->
+split-KV decode -> merge -> short decode rows: every row of the hot path.
+`value` is prefill tokens/s (B*N tokens per step) with inputs resident in HBM
+(3.7 GB of queries alone, far larger than the 126 MB L2, which is also flushed
+before every step by writing a 256 MiB buffer outside the timed events).  The
+default line also carries sub-records measured in the same run: the 4 x 1M
+decode over the packed rotated and the natural HND caches, and the
+Qwen2.5-0.5B-shaped 32K prefill line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --workload NAME ...
@@ -248,13 +252,14 @@ def run_sparse(args, wl):
                            l2="flushed before every step (256 MiB write, outside the timed events)"),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "traffic": None,
-                         "kernel": f"whole call: rope_pack(q), rope_pack(k), prefill_tc_kernel<{D}, block mask>",
+                         "kernel": f"whole call: rope_pack(q), rope_pack(k), prefill_tc_kernel<{D}, block mask>, "
+                                   "short rows",
                          "peak_source": f"{src} ({'sustained' if long_region else 'burst'} bf16)",
                          "flops_per_launch": flops},
             "window_off": {"ms_per_step": round(ms_off, 4)},
             "on_off_speedup": round(ms_off / ms, 4),
             "dense_window_on": {"ms_per_step": round(ms_dense, 4), "selection_speedup": round(ms_dense / ms, 4)},
-            "gpu_launches": 3 * args.steps, "clocks": clocks}
+            "gpu_launches": 4 * args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -274,18 +279,20 @@ VARLEN_WORKLOADS = {
                          "D": 128, "total": 1 << 20, "len_lo": 4096, "len_hi": 262144, "rope_base": 1e7,
                          "k_window": 16.0, "seed": 7},
 }
-WORKLOAD = WORKLOADS["qwen05b_32k"]
+DEFAULT_WORKLOAD = "qwen7b_512k"
+# Lines measured in the same run as the default one and reported inside it.
+SUB_RECORDS = ("decode_1m_packed", "decode_1m", "qwen05b_32k")
 L2_FLUSH_BYTES = 256 << 20
-KERNELS_PER_STEP = 5  # rope_pack(q), rope_pack(k), prefill_tc, decode_split, decode_merge
+# rope_pack(q), rope_pack(k), prefill_tc, short rows, decode_split, decode_merge, short decode rows
+KERNELS_PER_STEP = 7
 
-# DRAM bytes per launch of the tcgen05 prefill kernel on this workload, from one
-# ncu capture (profiles/prefill_tc_qwen05b_32k.md).  Valid only while the
-# kernel source hashes to `source_sha1`; otherwise the line reports null.
+# DRAM bytes per launch of the tcgen05 prefill kernel, from one ncu capture per
+# workload.  Valid only while the kernel source hashes to `source_sha1`;
+# otherwise the line reports null.
 TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98168320,
            "source_sha1": "fd039e524fa9ed078dfba5e3b08f3de1cb0a5392"}
 # DRAM bytes per launch of the decode kernel (split states included, merge not) on
-# the full-size workloads, from single-pass ncu captures
-# (profiles/decode_tc_qwen7b_packed_4x128k.md); valid while decode_tc.cu hashes to
+# the full-size workloads, from ncu captures; valid while decode_tc.cu hashes to
 # `source_sha1`.
 DECODE_TRAFFIC = {"decode_1m_packed": {"bytes_per_launch": 6607293952,
                                        "source_sha1": "61a5dcf9b9fce74f5022cf838de7d70f2150435d"},
@@ -296,12 +303,13 @@ DECODE_TRAFFIC = {"decode_1m_packed": {"bytes_per_launch": 6607293952,
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--workload", default="qwen05b_32k",
+    p.add_argument("--no-sub-records", action="store_true")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD,
                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(VARLEN_WORKLOADS) +
                    sorted(SPARSE_WORKLOADS))
     p.add_argument("--N", type=int, default=None, help="override sequence length (sweeps)")
@@ -441,31 +449,61 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- CPU oracle
-def cpu_baseline(q, k, v, wl, budget_s=12.0):
-    """The fp64 oracle, as it stands, on a bounded sample of query rows (all heads)."""
-    import contextlib
-    import numpy as np
-    import oracle
-    th = rope_theta(wl)
-    N = wl["N"]
-    kh = k[0].float().cpu().numpy()
-    vh = v[0].float().cpu().numpy()
-    rng = np.random.default_rng(1234)
+def oracle_rows_per_step(wl):
+    """Query rows (all heads) the oracle computes per step, one rule for both arms:
+    about 2^33 / (N * Hq * D) rows, so that a step is about a second of host work
+    whatever the workload (5 rows at the 512K default, 292 at 32K)."""
+    return max(1, round(2 ** 33 / (wl["N"] * wl["Hq"] * wl["D"])))
 
-    def run(nrows):
-        rows = np.sort(rng.choice(N, size=nrows, replace=False))
-        qh = q[0, rows].float().cpu().numpy()
-        t0 = time.perf_counter()
-        with (oracle.scaled_rope(th) if th is not None else contextlib.nullcontext()):
-            oracle.prefill_rows(qh, rows, kh, vh, wl["rope_base"], wl["k_window"])
-        return time.perf_counter() - t0
 
-    t = run(8)
-    nrows = int(max(8, min(N, 8 * budget_s / max(t, 1e-3))))
-    t = run(nrows)
-    return {"value": nrows / t, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
-            "sample": f"{nrows} uniformly drawn query rows x all {wl['Hq']} heads of the workload "
-                      f"(each row attends its full causal prefix), {t:.1f} s"}
+class OracleSample:
+    """The fp64 oracle, as it stands, on seeded uniformly drawn query rows of the
+    workload (every head; each row attends its full causal prefix)."""
+
+    def __init__(self, wl, k, v, q_rows):
+        import numpy as np
+        self.wl, self.k, self.v, self.q_rows = wl, k, v, q_rows
+        self.rows = oracle_rows_per_step(wl)
+        self.rng = np.random.default_rng(99)
+        self.th = rope_theta(wl)
+
+    def step(self):
+        import contextlib
+        import numpy as np
+        import oracle
+        rows = np.sort(self.rng.choice(self.wl["N"], size=self.rows, replace=False))
+        qr = self.q_rows(rows)
+        with (oracle.scaled_rope(self.th) if self.th is not None else contextlib.nullcontext()):
+            oracle.prefill_rows(qr, rows, self.k, self.v, self.wl["rope_base"], self.wl["k_window"])
+
+    def describe(self, steps, seconds):
+        import oracle
+        return {"value": steps * self.rows / seconds, "unit": "tokens/s", "cores": oracle.threads(),
+                "kind": "oracle",
+                "sample": f"{steps} steps of {self.rows} seeded uniformly drawn query rows x all {self.wl['Hq']} "
+                          f"heads (each row attends its full causal prefix), {seconds:.1f} s"}
+
+
+def cpu_baseline(q, k, v, wl, budget_s=10.0):
+    """The oracle timed on the host cores, on the reference arm's sampling rule."""
+    kh, vh = k[0].float().cpu().numpy(), v[0].float().cpu().numpy()
+    smp = OracleSample(wl, kh, vh, lambda rows: q[0, rows].float().cpu().numpy())
+    t0 = time.perf_counter()
+    smp.step()  # warm-up, also sizes the run
+    t1 = time.perf_counter() - t0
+    steps = max(3, min(50, int(budget_s / max(t1, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        smp.step()
+    return smp.describe(steps, time.perf_counter() - t0)
+
+
+def line_config(wl, world):
+    """The `config` of a prefill line; both arms report the same one."""
+    big = 2 * wl["B"] * wl["N"] * wl["Hq"] * wl["D"] > (126 << 20)
+    l2 = ("inputs larger than L2, which is also flushed before every step (256 MiB write, outside the timed "
+          "events)" if big else "flushed before every step (256 MiB write, outside the timed events)")
+    return dict(wl, l2=l2, parallelism="replicas" if world > 1 else "single GPU")
 
 
 def run_reference(args, wl):
@@ -473,57 +511,77 @@ def run_reference(args, wl):
     world, rank, _ = dist_setup()
     if rank != 0:
         return
-    import numpy as np
-    import oracle
     from long_context_attention_pair_b200 import synthetic
-    N, rows_per_step = wl["N"], 4
+    N = wl["N"]
     shape_kv = (wl["B"], N, wl["Hkv"], wl["D"])
     k = synthetic.tensor(wl["seed"], "k", shape_kv, "bf16")[0]
     v = synthetic.tensor(wl["seed"], "v", shape_kv, "bf16")[0]
-    rng = np.random.default_rng(99)
     qshape = (wl["B"], N, wl["Hq"], wl["D"])
-
-    th = rope_theta(wl)
-
-    def step():
-        rows = np.sort(rng.choice(N, size=rows_per_step, replace=False))
-        qr = synthetic.rows(wl["seed"], "q", qshape, 1, rows, "bf16")[0]
-        if th is None:
-            oracle.prefill_rows(qr, rows, k, v, wl["rope_base"], wl["k_window"])
-        else:
-            with oracle.scaled_rope(th):
-                oracle.prefill_rows(qr, rows, k, v, wl["rope_base"], wl["k_window"])
-
+    smp = OracleSample(wl, k, v, lambda rows: synthetic.rows(wl["seed"], "q", qshape, 1, rows, "bf16")[0])
     for _ in range(args.warmup):
-        step()
+        smp.step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        step()
+        smp.step()
     t = time.perf_counter() - t0
-    value = args.steps * rows_per_step / t
-    cb = {"value": value, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
-          "sample": f"{rows_per_step} random query rows x all heads per step"}
+    cb = smp.describe(args.steps, t)
+    value = cb["value"]
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": dict(wl), "cpu_baseline": cb,
+            "data": "synthetic", "config": line_config(wl, args.gpus), "cpu_baseline": cb,
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 # -------------------------------------------------------------------- our arm
-def run_ours(args, wl):
+def init_dist(local):
     import torch
-    import long_context_attention_pair_b200 as atf
-    from long_context_attention_pair_b200 import synthetic
-
-    world, rank, local = dist_setup()
+    world = dist_setup()[0]
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    return dev
+
+
+def finish_dist(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_ours(args, wl):
+    world, rank, local = dist_setup()
+    dev = init_dist(local)
+    line = measure_prefill(args, wl, args.workload, dev, e2e_on=not args.no_e2e,
+                           cpu_on=rank == 0 and world == 1 and not args.no_cpu_baseline)
+    if args.workload == DEFAULT_WORKLOAD and not args.no_sub_records and args.N is None and args.k_window is None:
+        import torch
+        subs = {}
+        torch.cuda.empty_cache()
+        for name in SUB_RECORDS:
+            if name in DECODE_WORKLOADS:
+                subs[name] = measure_decode(args, dict(DECODE_WORKLOADS[name]), name, dev)
+            else:
+                subs[name] = measure_prefill(args, dict(WORKLOADS[name]), name, dev, e2e_on=False, cpu_on=False)
+            torch.cuda.empty_cache()
+        line["sub_records"] = subs
+        line["gpu_launches"] += sum(r["gpu_launches"] for r in subs.values())
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    finish_dist(world)
+
+
+def measure_prefill(args, wl, name, dev, e2e_on, cpu_on):
+    """One prefill workload's line (every rank measures; times are max over ranks)."""
+    import torch
+    import long_context_attention_pair_b200 as atf
+    from long_context_attention_pair_b200 import synthetic
+
+    world, rank, local = dist_setup()
     B, N, Hq, Hkv, D = wl["B"], wl["N"], wl["Hq"], wl["Hkv"], wl["D"]
     base, kwin = wl["rope_base"], wl["k_window"]
     th = rope_theta(wl)
@@ -549,6 +607,7 @@ def run_ours(args, wl):
         atf.prefill_packed(qpack, kpack, v, base, kw, out=out, **tk)
         if ev is not None:
             ev[1].record(stream)
+        atf.prefill_short_rows(q, k, v, out, base, kw, **tk)
         atf.decode(q_last, k, v, seqlens, base, kw, kv_layout="NHD", out=dec_out, workspace=dws, **tk)
 
     def timed(kw, steps):
@@ -607,7 +666,7 @@ def run_ours(args, wl):
     long_region = total_ms > 2000.0
     peak = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
     achieved = flops / (kern_ms / 1e3) / 1e12
-    traffic = prefill_traffic(args.workload, wl)
+    traffic = prefill_traffic(name, wl)
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": f"prefill_tc_kernel<{D}>",
                 "kernel_ms": round(kern_ms, 4),
@@ -618,8 +677,7 @@ def run_ours(args, wl):
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(wl, l2="flushed before every step (256 MiB write, outside the timed events)",
-                       parallelism="replicas" if world > 1 else "single GPU"),
+        "config": line_config(wl, world),
         "roofline": roofline,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clocks,
@@ -633,15 +691,13 @@ def run_ours(args, wl):
         "median_step_ms": round(med_ms, 4),
     }
 
-    if not args.no_e2e:
+    if e2e_on:
+        del qpack, kpack, out, dws, flush
+        torch.cuda.empty_cache()
         line["e2e"] = e2e(atf, q, k, v, wl, args, dev, world)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if cpu_on:
         line["cpu_baseline"] = cpu_baseline(q, k, v, wl)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    return line
 
 
 def decode_retained_bytes(atf, wl):
@@ -656,16 +712,20 @@ def decode_retained_bytes(atf, wl):
 
 
 def run_decode(args, wl):
+    world, rank, local = dist_setup()
+    dev = init_dist(local)
+    line = measure_decode(args, wl, args.workload, dev)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    finish_dist(world)
+
+
+def measure_decode(args, wl, name, dev):
+    """One decode workload's line (every rank measures; times are max over ranks)."""
     import torch
     import long_context_attention_pair_b200 as atf
     from long_context_attention_pair_b200 import synthetic
     world, rank, local = dist_setup()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     B, Hq, Hkv, D, L = wl["B"], wl["Hq"], wl["Hkv"], wl["D"], wl["N"]
     base, kwin = wl["rope_base"], wl["k_window"]
     q = synthetic.tensor_torch(wl["seed"], "q_dec", (B, Hq, D), "bf16", device=dev)
@@ -742,16 +802,12 @@ def run_decode(args, wl):
             "config": dict(wl, l2="inputs larger than L2 (cache of %.1f GB)" % (2 * B * Hkv * L * D * 2 / 1e9)),
             "decode": {"us_per_call": round(1e3 * ms, 2), "us_per_token": round(1e3 * ms / B, 2)},
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": decode_traffic(args.workload, L),
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": decode_traffic(name, L),
                          "kernel": f"decode_tc_kernel<{D}{', paged' if page else ''}> + decode_merge_kernel",
                          "bytes_per_call": nbytes, "peak_source": src},
             "window_off": {"ms_per_step": round(ms_off, 4), "us_per_token": round(1e3 * ms_off / B, 2)},
-            "on_off_speedup": round(ms_off / ms, 4), "gpu_launches": 2 * args.steps, "clocks": clocks}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+            "on_off_speedup": round(ms_off / ms, 4), "gpu_launches": 3 * args.steps, "clocks": clocks}
+    return line
 
 
 def ragged_lengths(seed, total, lo, hi):
@@ -838,13 +894,14 @@ def run_varlen(args, wl):
                            l2="flushed before every step (256 MiB write, outside the timed events)"),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "traffic": None,
-                         "kernel": f"whole call: rope_pack(q), rope_pack(k), prefill_tc_kernel<{D}, varlen>",
+                         "kernel": f"whole call: rope_pack(q), rope_pack(k), prefill_tc_kernel<{D}, varlen>, "
+                                   "short rows",
                          "peak_source": f"{src} ({'sustained' if long_region else 'burst'} bf16)",
                          "flops_per_launch": flops},
             "window_off": {"ms_per_step": round(ms_off, 4), "value": round(world * total / (ms_off / 1e3), 1)},
             "on_off_speedup": round(ms_off / ms, 4),
             "pruned_fraction": round(pruned / all_terms, 6),
-            "gpu_launches": 3 * args.steps, "clocks": clocks}
+            "gpu_launches": 4 * args.steps, "clocks": clocks}
     if not args.no_e2e:
         line["e2e"] = e2e_varlen(atf, q, k, v, cu, max_len, wl, args, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

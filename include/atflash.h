@@ -49,6 +49,8 @@ typedef struct CUstream_st *cudaStream_t;
 #define ATFLASH_ERR_CUDA (-4)        /* a CUDA runtime/driver call or launch failed */
 #define ATFLASH_ERR_TIMEOUT (-5)     /* a kernel's bounded wait ran out (device status) */
 #define ATFLASH_ERR_ALIGNMENT (-6)   /* a pointer is not 16-byte aligned */
+#define ATFLASH_ERR_BAD_PAGE (-7)    /* a paged decode met a page index past its block-table row or a
+                                        page id outside the pool (device status) */
 
 /* Element types of tensors passed to the GPU calls. */
 #define ATFLASH_F32 0
@@ -131,6 +133,30 @@ int atflash_prefill_ex(const void *q, const void *k, const void *v, void *out, i
                        int Hkv, int64_t N, int D, double rope_base, double k_window, int in_dtype,
                        int out_dtype, float *lse, void *workspace, size_t workspace_bytes,
                        cudaStream_t stream);
+
+/*
+ * Accuracy of short rows.  The tensor-core path rounds the rotated queries and
+ * keys, and the probabilities P, to bf16.  Over a row that sees few keys those
+ * roundings do not average out (seeded sweeps measured errors up to 1.06e-2 on
+ * rows of 4-16 keys, against below 4e-3 on rows of more than 128 keys), so
+ * every bf16 call recomputes, after its tensor-core kernel, each row that sees
+ * at most 128 keys in fp32 on CUDA cores from the un-rotated inputs, by the
+ * method's plain definition ("The idea": RoPE, the per-pair window, softmax,
+ * P.V), and overwrites that row's output and log-sum-exp: the first 128-row
+ * tile of every prefill sequence, every query tile of a block selection whose
+ * mask selects no earlier key tile, and every decode sequence of at most 128
+ * tokens.
+ *
+ * atflash_prefill_short_rows is that step on its own, for callers that run
+ * atflash_rope_pack + atflash_prefill_packed themselves: same q, k, v (the
+ * un-rotated bf16 inputs), out, out_dtype, lse, shapes and errors as
+ * atflash_prefill_ex with in_dtype ATFLASH_BF16; queue it after the packed
+ * prefill on the same stream.  The three calls together give the same bits as
+ * atflash_prefill_ex.
+ */
+int atflash_prefill_short_rows(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
+                               int64_t N, int D, double rope_base, double k_window, int out_dtype, float *lse,
+                               cudaStream_t stream);
 
 /*
  * Windowed prefill on top of a token-level block selection ("Abstract": token-
@@ -218,7 +244,10 @@ size_t atflash_prefill_varlen_workspace_bytes(int Hq, int Hkv, int64_t total, in
  *               vpages as for NHD.
  *   block_table device int32 [B][max_pages]; seqlens device int32 [B],
  *               1 <= seqlens[b] <= max_pages*page_size.  A page index past
- *               the row or an id outside [0, num_pages) reads zeros.
+ *               the row or an id outside [0, num_pages) is an error found on
+ *               the device: the kernel records ATFLASH_ERR_BAD_PAGE in the
+ *               device status word (atflash_device_status) and reads zeros in
+ *               its place, so that sequence's output is not valid.
  *   workspace   >= atflash_decode_workspace_bytes(B, Hq, Hkv,
  *               max_pages*page_size, D) bytes, 16-byte aligned.
  * Errors as atflash_decode, plus ATFLASH_ERR_INVALID_ARG for page_size,
@@ -282,6 +311,9 @@ int atflash_prefill_sparse_theta(const void *q, const void *k, const void *v, co
                                  void *out, int B, int Hq, int Hkv, int64_t N, int D, const double *theta,
                                  double k_window, int out_dtype, float *lse, void *workspace,
                                  size_t workspace_bytes, cudaStream_t stream);
+int atflash_prefill_short_rows_theta(const void *q, const void *k, const void *v, void *out, int B, int Hq,
+                                     int Hkv, int64_t N, int D, const double *theta, double k_window, int out_dtype,
+                                     float *lse, cudaStream_t stream);
 /* qpack/kpack written by atflash_rope_pack_theta with the same table. */
 int atflash_prefill_packed_theta(const void *qpack, const void *kpack, const void *v, void *out, int B, int Hq,
                                  int Hkv, int64_t N, int D, const double *theta, double k_window, int in_dtype,
@@ -310,10 +342,16 @@ int atflash_decode_paged_theta(const void *q, const void *kpages, const void *vp
  * every GPU loading the library reserves until the process exits.
  *   Returns ATFLASH_ERR_WORKSPACE, launching nothing, when the problem needs
  *   more than that (atflash_decode_workspace_bytes() > the limit).
+ *   The array is part of the library's device image: every process that loads
+ *   the library holds these 32 MiB on every GPU it uses, whether or not it
+ *   calls this entry point.
+ *   Arguments are checked exactly as atflash_decode checks them (same status
+ *   for the same bad argument).
  *   Every call on a device shares the array: calls whose work overlaps on the
  *   GPU race; calls on one stream are ordered.  The first call on a device
- *   looks up the array's address with that device current; make it before any
- *   stream capture begins.
+ *   looks up the array's address with that device current and keeps it; make
+ *   it before any stream capture begins, and do not reset the device
+ *   (cudaDeviceReset) after it.
  */
 #define ATFLASH_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 int atflash_decode_noalloc(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens,
@@ -322,9 +360,10 @@ int atflash_decode_noalloc(const void *q, const void *kcache, const void *vcache
                            cudaStream_t stream);
 
 /*
- * Device status word of the current device: ATFLASH_OK, or ATFLASH_ERR_TIMEOUT
- * when a kernel's bounded wait ran out since the last clear.  Synchronises
- * the device.  clear != 0 resets the word.
+ * Device status word of the current device: ATFLASH_OK, ATFLASH_ERR_TIMEOUT
+ * when a kernel's bounded wait ran out, or ATFLASH_ERR_BAD_PAGE when a paged
+ * decode met a bad page index, since the last clear (the first such event is
+ * kept).  Synchronises the device.  clear != 0 resets the word.
  */
 int atflash_device_status(int clear);
 

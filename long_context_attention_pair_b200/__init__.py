@@ -18,7 +18,7 @@ import os
 __all__ = [
     "lib", "prefill", "decode", "pruned_terms", "window_table", "prefill_workspace_bytes",
     "decode_workspace_bytes", "device_status", "AtflashError", "F32", "BF16", "rope_pack", "prefill_packed",
-    "prefill_bf16", "theta_table", "prefill_sparse",
+    "prefill_bf16", "theta_table", "prefill_sparse", "prefill_short_rows",
 ]
 
 F32 = 0
@@ -28,6 +28,7 @@ KV_NHD = 1
 KV_PACKED = 2
 OK = 0
 ERR_TIMEOUT = -5
+ERR_BAD_PAGE = -7
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libatflash.so")
@@ -88,13 +89,16 @@ def lib():
         L.atflash_prefill_packed_theta.argtypes = [vp, vp, vp, vp, i, i, i, i64, i, dp, d, i, i, vp, vp]
         L.atflash_prefill_sparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i64, i, d, d, i, vp, vp, sz, vp]
         L.atflash_prefill_sparse_theta.argtypes = [vp, vp, vp, vp, vp, i, i, i, i64, i, dp, d, i, vp, vp, sz, vp]
+        L.atflash_prefill_short_rows.argtypes = [vp, vp, vp, vp, i, i, i, i64, i, d, d, i, vp, vp]
+        L.atflash_prefill_short_rows_theta.argtypes = [vp, vp, vp, vp, i, i, i, i64, i, dp, d, i, vp, vp]
         for f in ("atflash_window_table", "atflash_pruned_terms", "atflash_prefill", "atflash_prefill_ex",
                   "atflash_decode", "atflash_device_status", "atflash_rope_pack", "atflash_prefill_packed",
                   "atflash_prefill_varlen", "atflash_decode_paged", "atflash_theta_table",
                   "atflash_window_table_theta", "atflash_pruned_terms_theta", "atflash_rope_pack_theta",
                   "atflash_prefill_theta", "atflash_decode_theta", "atflash_prefill_varlen_theta",
                   "atflash_decode_paged_theta", "atflash_prefill_packed_theta", "atflash_prefill_sparse",
-                  "atflash_prefill_sparse_theta"):
+                  "atflash_prefill_sparse_theta", "atflash_prefill_short_rows",
+                  "atflash_prefill_short_rows_theta"):
             getattr(L, f).restype = i
         _lib = L
     return _lib
@@ -366,6 +370,24 @@ def prefill_packed(qpack, kpack, v, rope_base: float, k_window: float = math.inf
     return out
 
 
+def prefill_short_rows(q, k, v, out, rope_base: float, k_window: float = math.inf, *, lse=None, stream=None,
+                       theta=None):
+    """The short-row step on its own: recompute in fp32 the rows that see at most
+    128 keys (the first 128-row tile of every sequence) from the un-rotated bf16
+    q [B, N, Hq, D], k/v [B, N, Hkv, D], overwriting them in ``out`` (and ``lse``
+    [B, Hq, N]).  Queue it after ``prefill_packed`` on the same stream; the
+    three steps then give the bits of ``prefill``."""
+    B, N, Hq, D = q.shape
+    fn, name, rope = lib().atflash_prefill_short_rows, "atflash_prefill_short_rows", float(rope_base)
+    if theta is not None:
+        fn, name, rope = (lib().atflash_prefill_short_rows_theta, "atflash_prefill_short_rows_theta",
+                          _theta_arg(theta, D))
+    st = fn(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), B, Hq, k.shape[2], N, D, rope,
+            float(k_window), _dtype_code(out), _dev(lse, "lse") if lse is not None else None, _stream_ptr(stream))
+    _check(st, name)
+    return out
+
+
 def prefill_bf16(q, k, v, out, rope_base: float, k_window: float = math.inf, stream=None):
     """The plain bf16 call (library-managed scratch), writing into ``out``."""
     B, N, Hq, D = q.shape
@@ -419,7 +441,8 @@ def decode(q, k_cache, v_cache, seqlens, rope_base: float, k_window: float = mat
 
 
 def device_status(clear: bool = True) -> int:
-    """ATFlash device status word (0, or -5 after a kernel's bounded wait ran out)."""
+    """ATFlash device status word: 0, -5 after a kernel's bounded wait ran out, or
+    -7 after a paged decode met a bad page index (the first event is kept)."""
     return int(lib().atflash_device_status(1 if clear else 0))
 
 

@@ -124,6 +124,66 @@ static size_t prefill_ws(int B, int Hq, int Hkv, int64_t N, int D, int in_dtype)
     return align256((size_t)B * Hq * N * D * es) + align256((size_t)B * Hkv * N * D * es);
 }
 
+// theta_r = base^(-2r/D) after the same checks as the base-taking calls.
+int theta_from_base(int D, double base, double *theta) {
+    const int rc = check_window_args(D, base, 0.0);
+    if (rc == ATFLASH_OK) theta_table(D, base, theta);
+    return rc;
+}
+
+// atflash_decode's argument checks; on success the scratch it needs (need) is
+// known but not yet checked.  Shared by atflash_decode and the entry point that
+// allocates nothing, so that both reject the same arguments the same way.
+int decode_check(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out, int B,
+                 int Hq, int Hkv, int64_t Nmax, int D, const double *theta, double k_window, int kcache_rotated,
+                 int kv_layout, int in_dtype, int out_dtype, size_t *need) {
+    if (!q || !kcache || !vcache || !seqlens || !out) return ATFLASH_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, Nmax);
+    if (rc != ATFLASH_OK) return rc;
+    if ((rc = check_theta_args(D, theta, k_window)) != ATFLASH_OK) return rc;
+    if (kcache_rotated != 0 && kcache_rotated != 1) return ATFLASH_ERR_INVALID_ARG;
+    if (kv_layout != ATFLASH_KV_HND && kv_layout != ATFLASH_KV_NHD && kv_layout != ATFLASH_KV_PACKED)
+        return ATFLASH_ERR_INVALID_ARG;
+    if (kv_layout == ATFLASH_KV_PACKED && !kcache_rotated) return ATFLASH_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
+    if ((in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) ||
+        (out_dtype != ATFLASH_F32 && out_dtype != ATFLASH_BF16))
+        return ATFLASH_ERR_UNSUPPORTED;
+    if (Hq / Hkv > 16) return ATFLASH_ERR_UNSUPPORTED;
+    if (kv_layout == ATFLASH_KV_PACKED && in_dtype != ATFLASH_BF16) return ATFLASH_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out))
+        return ATFLASH_ERR_ALIGNMENT;
+    *need = decode_workspace_bytes(B, Hq, Hkv, Nmax, D);
+    return ATFLASH_OK;
+}
+
+// The decode after decode_check, into a workspace of at least its `need` bytes.
+int decode_run(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out, int B,
+               int Hq, int Hkv, int64_t Nmax, int D, const double *theta, double k_window, int kcache_rotated,
+               int kv_layout, int in_dtype, int out_dtype, float *workspace, cudaStream_t stream) {
+    WindowParams wp;
+    int rc = fill_window_theta(wp, D, theta, k_window, Nmax);
+    if (rc != ATFLASH_OK) return rc;
+    Problem p{B, Hq, Hkv, D, Nmax};
+    cudaError_t e = launch_decode(q, kcache, vcache, seqlens, out, out_dtype == ATFLASH_F32,
+                                  in_dtype == ATFLASH_F32, kcache_rotated, kv_layout, p, wp, workspace, stream);
+    return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
+}
+
+static int decode_impl(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out,
+                       int B, int Hq, int Hkv, int64_t Nmax, int D, const double *theta, double k_window,
+                       int kcache_rotated, int kv_layout, int in_dtype, int out_dtype, void *workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
+    size_t need = 0;
+    int rc = decode_check(q, kcache, vcache, seqlens, out, B, Hq, Hkv, Nmax, D, theta, k_window, kcache_rotated,
+                          kv_layout, in_dtype, out_dtype, &need);
+    if (rc != ATFLASH_OK) return rc;
+    if (!workspace || workspace_bytes < need) return ATFLASH_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return ATFLASH_ERR_ALIGNMENT;
+    return decode_run(q, kcache, vcache, seqlens, out, B, Hq, Hkv, Nmax, D, theta, k_window, kcache_rotated,
+                      kv_layout, in_dtype, out_dtype, static_cast<float *>(workspace), stream);
+}
+
 }  // namespace atf
 
 using namespace atf;
@@ -139,6 +199,7 @@ const char *atflash_status_string(int status) {
         case ATFLASH_ERR_CUDA: return "CUDA runtime or launch error";
         case ATFLASH_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
         case ATFLASH_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case ATFLASH_ERR_BAD_PAGE: return "a paged decode met a page index outside its block table or pool";
         default: return "unknown status";
     }
 }
@@ -218,6 +279,23 @@ static int run_rope_pack(const void *x, void *y, int B, int64_t N, int H, int D,
     for (int r = 0; r < D / 2; ++r) wp.theta[r] = theta[r];
     cudaError_t e = (in_dtype == ATFLASH_BF16) ? launch_rope_pack_bf16(x, y, B, N, H, D, wp, stream)
                                                : launch_rope_pack_f32(x, y, B, N, H, D, wp, stream);
+    return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
+}
+
+// The rows that see at most 128 keys, recomputed in fp32 from the caller's
+// un-rotated bf16 inputs after the tensor-core prefill (see short_rows.cu).
+static int run_short_rows(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv, int64_t N,
+                          int D, const double *theta, double k_window, int out_dtype, float *lse,
+                          cudaStream_t stream, const int32_t *cu_seqlens = nullptr, int64_t total = 0,
+                          const uint8_t *block_mask = nullptr) {
+    WindowParams wp;
+    int rc = fill_window_theta(wp, D, theta, k_window, N);
+    if (rc != ATFLASH_OK) return rc;
+    int *status = device_status_word();
+    if (!status) return ATFLASH_ERR_CUDA;
+    Problem p{B, Hq, Hkv, D, N};
+    cudaError_t e = launch_short_rows_prefill(q, k, v, out, out_dtype == ATFLASH_F32, lse, p, wp, status, stream,
+                                              cu_seqlens, total, block_mask);
     return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
 }
 
@@ -307,7 +385,9 @@ static int prefill_ex_impl(const void *q, const void *k, const void *v, void *ou
     void *kt = ws + align256((size_t)B * Hq * N * D * es);
     if ((rc = run_rope_pack(q, qt, B, N, Hq, D, theta, in_dtype, stream)) != ATFLASH_OK) return rc;
     if ((rc = run_rope_pack(k, kt, B, N, Hkv, D, theta, in_dtype, stream)) != ATFLASH_OK) return rc;
-    return run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, theta, k_window, in_dtype, out_dtype, lse, stream);
+    rc = run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, theta, k_window, in_dtype, out_dtype, lse, stream);
+    if (rc != ATFLASH_OK || in_dtype != ATFLASH_BF16) return rc;
+    return run_short_rows(q, k, v, out, B, Hq, Hkv, N, D, theta, k_window, out_dtype, lse, stream);
 }
 
 static int prefill_sparse_impl(const void *q, const void *k, const void *v, const uint8_t *block_mask, void *out,
@@ -325,8 +405,11 @@ static int prefill_sparse_impl(const void *q, const void *k, const void *v, cons
     void *kt = ws + align256((size_t)B * Hq * N * D * 2);
     if ((rc = run_rope_pack(q, qt, B, N, Hq, D, theta, ATFLASH_BF16, stream)) != ATFLASH_OK) return rc;
     if ((rc = run_rope_pack(k, kt, B, N, Hkv, D, theta, ATFLASH_BF16, stream)) != ATFLASH_OK) return rc;
-    return run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, theta, k_window, ATFLASH_BF16, out_dtype, lse,
-                              stream, block_mask);
+    rc = run_prefill_packed(qt, kt, v, out, B, Hq, Hkv, N, D, theta, k_window, ATFLASH_BF16, out_dtype, lse, stream,
+                            block_mask);
+    if (rc != ATFLASH_OK) return rc;
+    return run_short_rows(q, k, v, out, B, Hq, Hkv, N, D, theta, k_window, out_dtype, lse, stream, nullptr, 0,
+                          block_mask);
 }
 
 int atflash_prefill_sparse(const void *q, const void *k, const void *v, const uint8_t *block_mask, void *out,
@@ -347,6 +430,31 @@ int atflash_prefill_sparse_theta(const void *q, const void *k, const void *v, co
     if (!q || !k || !v || !out || !block_mask) return ATFLASH_ERR_INVALID_ARG;
     return prefill_sparse_impl(q, k, v, block_mask, out, B, Hq, Hkv, N, D, theta, k_window, out_dtype, lse,
                                workspace, workspace_bytes, stream);
+}
+
+static int short_rows_impl(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
+                           int64_t N, int D, const double *theta, double k_window, int out_dtype, float *lse,
+                           cudaStream_t stream) {
+    if (!q || !k || !v || !out) return ATFLASH_ERR_INVALID_ARG;
+    int rc = check_prefill_common(B, Hq, Hkv, N, D, theta, k_window, ATFLASH_BF16, out_dtype);
+    if (rc != ATFLASH_OK) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATFLASH_ERR_ALIGNMENT;
+    return run_short_rows(q, k, v, out, B, Hq, Hkv, N, D, theta, k_window, out_dtype, lse, stream);
+}
+
+int atflash_prefill_short_rows(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
+                               int64_t N, int D, double rope_base, double k_window, int out_dtype, float *lse,
+                               cudaStream_t stream) {
+    if (!q || !k || !v || !out) return ATFLASH_ERR_INVALID_ARG;
+    BaseTheta bt(D, rope_base);
+    if (bt.rc != ATFLASH_OK) return bt.rc;
+    return short_rows_impl(q, k, v, out, B, Hq, Hkv, N, D, bt.theta, k_window, out_dtype, lse, stream);
+}
+
+int atflash_prefill_short_rows_theta(const void *q, const void *k, const void *v, void *out, int B, int Hq,
+                                     int Hkv, int64_t N, int D, const double *theta, double k_window, int out_dtype,
+                                     float *lse, cudaStream_t stream) {
+    return short_rows_impl(q, k, v, out, B, Hq, Hkv, N, D, theta, k_window, out_dtype, lse, stream);
 }
 
 int atflash_prefill_ex(const void *q, const void *k, const void *v, void *out, int B, int Hq, int Hkv,
@@ -435,6 +543,9 @@ static int prefill_varlen_impl(const void *q, const void *k, const void *v, void
         if (e == cudaSuccess)
             e = launch_prefill_tc(qt, kt, v, out, out_dtype == ATFLASH_F32, lse, p, wp, status, wait_limit_ns(),
                                   stream, cu_seqlens, total);
+        if (e == cudaSuccess)
+            e = launch_short_rows_prefill(q, k, v, out, out_dtype == ATFLASH_F32, lse, p, wp, status, stream,
+                                          cu_seqlens, total);
         if (e != cudaSuccess) rc = ATFLASH_ERR_CUDA;
     }
     if (owned) cudaFreeAsync(owned, stream);
@@ -518,38 +629,6 @@ int atflash_decode_paged_theta(const void *q, const void *kpages, const void *vp
                              workspace_bytes, stream);
 }
 
-static int decode_impl(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out,
-                       int B, int Hq, int Hkv, int64_t Nmax, int D, const double *theta, double k_window,
-                       int kcache_rotated, int kv_layout, int in_dtype, int out_dtype, void *workspace,
-                       size_t workspace_bytes, cudaStream_t stream) {
-    if (!q || !kcache || !vcache || !seqlens || !out) return ATFLASH_ERR_INVALID_ARG;
-    int rc = check_shape(B, Hq, Hkv, Nmax);
-    if (rc != ATFLASH_OK) return rc;
-    if ((rc = check_theta_args(D, theta, k_window)) != ATFLASH_OK) return rc;
-    if (kcache_rotated != 0 && kcache_rotated != 1) return ATFLASH_ERR_INVALID_ARG;
-    if (kv_layout != ATFLASH_KV_HND && kv_layout != ATFLASH_KV_NHD && kv_layout != ATFLASH_KV_PACKED)
-        return ATFLASH_ERR_INVALID_ARG;
-    if (kv_layout == ATFLASH_KV_PACKED && !kcache_rotated) return ATFLASH_ERR_INVALID_ARG;
-    if (D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
-    if ((in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) ||
-        (out_dtype != ATFLASH_F32 && out_dtype != ATFLASH_BF16))
-        return ATFLASH_ERR_UNSUPPORTED;
-    if (Hq / Hkv > 16) return ATFLASH_ERR_UNSUPPORTED;
-    if (kv_layout == ATFLASH_KV_PACKED && in_dtype != ATFLASH_BF16) return ATFLASH_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out))
-        return ATFLASH_ERR_ALIGNMENT;
-    const size_t need = decode_workspace_bytes(B, Hq, Hkv, Nmax, D);
-    if (!workspace || workspace_bytes < need) return ATFLASH_ERR_WORKSPACE;
-    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return ATFLASH_ERR_ALIGNMENT;
-    WindowParams wp;
-    if ((rc = fill_window_theta(wp, D, theta, k_window, Nmax)) != ATFLASH_OK) return rc;
-    Problem p{B, Hq, Hkv, D, Nmax};
-    cudaError_t e = launch_decode(q, kcache, vcache, seqlens, out, out_dtype == ATFLASH_F32,
-                                  in_dtype == ATFLASH_F32, kcache_rotated, kv_layout, p, wp,
-                                  static_cast<float *>(workspace), stream);
-    return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
-}
-
 int atflash_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out,
                    int B, int Hq, int Hkv, int64_t Nmax, int D, double rope_base, double k_window,
                    int kcache_rotated, int kv_layout, int in_dtype, int out_dtype, void *workspace,
@@ -577,6 +656,7 @@ int atflash_device_status(int clear) {
         int z = 0;
         if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(int)) != cudaSuccess) return ATFLASH_ERR_CUDA;
     }
+    if (v >= ATFLASH_DEVICE_BAD_PAGE) return ATFLASH_ERR_BAD_PAGE;
     return v >= ATFLASH_DEVICE_TIMEOUT_BASE ? ATFLASH_ERR_TIMEOUT : ATFLASH_OK;
 }
 

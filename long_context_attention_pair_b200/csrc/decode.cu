@@ -280,7 +280,11 @@ cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const i
     if (e != cudaSuccess) return e;
     decode_merge_kernel<<<dim3((unsigned)p.Hq, (unsigned)p.B, (unsigned)(p.D / kMergeDims)), kMergeThreads, 0, s>>>(
         workspace, out, out_f32, p.Hq, nsplit, p.D);
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess || in_f32) return e;
+    // bf16 caches: sequences of at most 128 tokens again in fp32 (the fp32 path is exact already).
+    int *status = device_status_word();
+    if (!status) return cudaErrorUnknown;
+    return launch_short_rows_decode(q, kc, vc, seqlens, out, out_f32, krot, layout, p, wp, status, s, paged);
 }
 
 }  // namespace atf

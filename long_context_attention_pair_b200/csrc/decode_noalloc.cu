@@ -13,14 +13,20 @@
 // Limits and rules of use:
 //  - the split states must fit in ATFLASH_NOALLOC_SCRATCH_BYTES; larger
 //    problems are rejected with ATFLASH_ERR_WORKSPACE before anything runs;
+//  - the array is part of the library's device image, so every process that
+//    loads the library holds its 32 MiB on every GPU it uses, whether or not it
+//    ever calls this entry point;
 //  - every call on a device shares the one array, so two calls whose work
 //    overlaps on the GPU (different streams without ordering between them)
 //    race on it; calls queued on one stream are ordered and safe;
 //  - the first call on a device looks up the array's device address once
-//    (with that device current); make that first call before any stream
-//    capture begins.
-// The array keeps the last call's contents.  Nothing in it needs to start at
-// zero: the split kernel writes every state the merge kernel reads.
+//    (with that device current) and keeps it; make that first call before any
+//    stream capture begins, and do not reset the device (cudaDeviceReset)
+//    after it, since the kept address would then be stale.
+// Arguments are checked by the same code as atflash_decode's (decode_check), so
+// both reject the same arguments with the same status.  The array keeps the
+// last call's contents.  Nothing in it needs to start at zero: the split kernel
+// writes every state the merge kernel reads.
 #include <math.h>
 #include <stdint.h>
 
@@ -56,8 +62,6 @@ int scratch_on_current_device(float **out) {
     return ATFLASH_OK;
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 }  // namespace atf
 
@@ -68,35 +72,16 @@ extern "C" int atflash_decode_noalloc(const void *q, const void *kcache, const v
                                       int D, double rope_base, double k_window, int kcache_rotated, int kv_layout,
                                       int in_dtype, int out_dtype, cudaStream_t stream) {
     if (!q || !kcache || !vcache || !seqlens || !out) return ATFLASH_ERR_INVALID_ARG;
-    if (B < 1 || Hq < 1 || Hkv < 1 || Nmax < 1 || Nmax > INT32_MAX || Hq % Hkv != 0) return ATFLASH_ERR_INVALID_ARG;
-    if ((int64_t)B * Hq > 65535 || !(rope_base > 1.0) || isnan(k_window) || k_window < 0.0)
-        return ATFLASH_ERR_INVALID_ARG;
-    if (kcache_rotated != 0 && kcache_rotated != 1) return ATFLASH_ERR_INVALID_ARG;
-    if (kv_layout != ATFLASH_KV_HND && kv_layout != ATFLASH_KV_NHD && kv_layout != ATFLASH_KV_PACKED)
-        return ATFLASH_ERR_INVALID_ARG;
-    if (kv_layout == ATFLASH_KV_PACKED && (!kcache_rotated || in_dtype != ATFLASH_BF16))
-        return ATFLASH_ERR_INVALID_ARG;
-    if (D != 64 && D != 128) return ATFLASH_ERR_UNSUPPORTED;
-    if ((in_dtype != ATFLASH_F32 && in_dtype != ATFLASH_BF16) ||
-        (out_dtype != ATFLASH_F32 && out_dtype != ATFLASH_BF16))
-        return ATFLASH_ERR_UNSUPPORTED;
-    if (Hq / Hkv > 16) return ATFLASH_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out)) return ATFLASH_ERR_ALIGNMENT;
-    if (decode_workspace_bytes(B, Hq, Hkv, Nmax, D) > kScratchBytes) return ATFLASH_ERR_WORKSPACE;
-
-    WindowParams wp;
-    int64_t w[kMaxPairs];
-    int rc = window_table(D, rope_base, k_window, Nmax, w);
+    double theta[kMaxPairs];
+    int rc = theta_from_base(D, rope_base, theta);
     if (rc != ATFLASH_OK) return rc;
-    memset(&wp, 0, sizeof(wp));
-    wp.H = D / 2;
-    for (int r = 0; r < D / 2; ++r) wp.w[r] = (int32_t)w[r];
-    theta_table(D, rope_base, wp.theta);
-
+    size_t need = 0;
+    rc = decode_check(q, kcache, vcache, seqlens, out, B, Hq, Hkv, Nmax, D, theta, k_window, kcache_rotated,
+                      kv_layout, in_dtype, out_dtype, &need);
+    if (rc != ATFLASH_OK) return rc;
+    if (need > kScratchBytes) return ATFLASH_ERR_WORKSPACE;
     float *scratch = nullptr;
     if ((rc = scratch_on_current_device(&scratch)) != ATFLASH_OK) return rc;
-    Problem p{B, Hq, Hkv, D, Nmax};
-    cudaError_t e = launch_decode(q, kcache, vcache, seqlens, out, out_dtype == ATFLASH_F32,
-                                  in_dtype == ATFLASH_F32, kcache_rotated, kv_layout, p, wp, scratch, stream);
-    return e == cudaSuccess ? ATFLASH_OK : ATFLASH_ERR_CUDA;
+    return decode_run(q, kcache, vcache, seqlens, out, B, Hq, Hkv, Nmax, D, theta, k_window, kcache_rotated,
+                      kv_layout, in_dtype, out_dtype, scratch, stream);
 }

@@ -244,11 +244,15 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
                 uint8_t *kst = sK + st * F::KBytes;
                 if constexpr (kPaged) {
                     // A stage never straddles a page (page_size is a multiple of 64).  A
-                    // page index past the table row or an id outside the pool becomes -1,
-                    // which the maps treat as out of bounds (zero fill, no access).
+                    // page index past the table row or an id outside the pool is reported
+                    // in the device status word and becomes -1, which the maps treat as
+                    // out of bounds (zero fill, no access).
                     const int64_t pi = k0 / page_size;
                     int page = pi < max_pages ? block_table[(size_t)b * max_pages + pi] : -1;
-                    if (page < 0 || page >= num_pages) page = -1;
+                    if (page < 0 || page >= num_pages) {
+                        atomicCAS(status, 0, ATFLASH_DEVICE_BAD_PAGE);
+                        page = -1;
+                    }
                     const int kk = (int)(k0 % page_size);
                     if (kPacked) {
                         // Pages hold a multiple of 64 keys, so the 128-byte row view always applies.

@@ -57,20 +57,54 @@ cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *
                               uint64_t wait_limit_ns, cudaStream_t s, const int32_t *cu_seqlens = nullptr,
                               int64_t total = 0, const uint8_t *block_mask = nullptr);
 
-// Split-KV decode + merge.
-int decode_split_keys(int B, int Hkv, int64_t Nmax);
-int decode_num_splits(int B, int Hkv, int64_t Nmax);
-size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D);
 // A paged KV cache: keys i*page_size.. of sequence b are in pool page
 // block_table[b*max_pages + i]; page_size is a multiple of 64.
 struct PagedKV {
     const int32_t *block_table;  // device, [B][max_pages]
     int max_pages, page_size, num_pages;
 };
+
+// Rows that see at most 128 keys, recomputed in fp32 on CUDA cores from the
+// caller's un-rotated bf16 q, k, v after the tensor-core kernel (short_rows.cu):
+// the first 128-row tile of every sequence, or with a block mask every query
+// tile whose mask row selects no earlier key tile.  Overwrites those rows of out
+// (and lse).  q/k/v/out/lse/cu_seqlens/block_mask as for launch_prefill_tc, with
+// the caller's natural q, k instead of the packed ones.
+cudaError_t launch_short_rows_prefill(const void *q, const void *k, const void *v, void *out, int out_f32,
+                                      float *lse, const Problem &p, const WindowParams &wp, int *status,
+                                      cudaStream_t s, const int32_t *cu_seqlens = nullptr, int64_t total = 0,
+                                      const uint8_t *block_mask = nullptr);
+// The same for a bf16 decode: every sequence of at most 128 tokens, recomputed
+// in fp32 after the merge (any cache layout, contiguous or paged).
+cudaError_t launch_short_rows_decode(const void *q, const void *kc, const void *vc, const int32_t *seqlens,
+                                     void *out, int out_f32, int krot, int layout, const Problem &p,
+                                     const WindowParams &wp, int *status, cudaStream_t s,
+                                     const PagedKV *paged = nullptr);
+
+// Split-KV decode + merge.
+int decode_split_keys(int B, int Hkv, int64_t Nmax);
+int decode_num_splits(int B, int Hkv, int64_t Nmax);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D);
+
 cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, const int32_t *seqlens, int krot,
                              int layout, const Problem &p, const WindowParams &wp, float *workspace, int split_keys,
                              int nsplit, int *status, uint64_t limit_ns, cudaStream_t s,
                              const PagedKV *paged = nullptr);
+
+// theta_r = base^(-2r/D) into theta (D/2 entries) after the base-taking calls'
+// checks (even D in 2..256, base > 1); ATFLASH_ERR_INVALID_ARG otherwise.
+int theta_from_base(int D, double base, double *theta);
+
+// atflash_decode in two halves (api.cu): decode_check validates the arguments
+// exactly as atflash_decode does and reports the scratch bytes the call needs;
+// decode_run builds the window table and launches into a workspace of at least
+// that size.  theta: host table of D/2 frequencies.
+int decode_check(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out, int B,
+                 int Hq, int Hkv, int64_t Nmax, int D, const double *theta, double k_window, int kcache_rotated,
+                 int kv_layout, int in_dtype, int out_dtype, size_t *need);
+int decode_run(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *out, int B,
+               int Hq, int Hkv, int64_t Nmax, int D, const double *theta, double k_window, int kcache_rotated,
+               int kv_layout, int in_dtype, int out_dtype, float *workspace, cudaStream_t stream);
 
 // Device status word of the current device (bounded waits record timeouts
 // here) and the wait limit in nanoseconds.

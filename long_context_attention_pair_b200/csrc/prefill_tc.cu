@@ -60,10 +60,6 @@ struct Warps {
 };
 constexpr uint32_t kChunkBytes = kBN * 32;  // 128 rows x 16 bf16 (one K-step)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
-// Of every 8 element pairs of a softmax row, this many take exp2 on the FMA
-// pipe (polynomial) and the rest on the multi-function unit, so that neither
-// unit alone bounds the softmax.
-constexpr int kPolyPairsOf8 = 0;
 // Boundary pairs whose key values the fix-up warp stages per tile (fp32, two
 // keys per 16 bytes); a tile with more boundary pairs handles the rest directly
 // from the K~ chunk.
@@ -95,7 +91,6 @@ struct Cfg {
     static constexpr uint32_t TmemCols = NH == 2 ? 512 : 256;
     static constexpr uint32_t TmemO0 = NH == 2 ? 256 : 128, TmemO1 = 256 + D;
     static constexpr bool SharedS = (D == 128);
-    static constexpr bool Token = false;  // alternate the two heads' exp2 passes (measured slower)
     static constexpr uint32_t TmemS0 = 0, TmemS1 = SharedS ? 0 : 128;
     static constexpr uint32_t TmemP0 = NH == 1 ? 192 : (SharedS ? 128 : 384), TmemP1 = SharedS ? 192 : 448;
 };
@@ -107,7 +102,6 @@ struct Ctl {
     uint64_t v_full[VS], v_empty[VS];
     uint64_t s_full[2], s_read[2], p_full[2], o_done[2];
     uint64_t drain;
-    uint64_t tok[2][4];  // [head][warp of the head]: that warp finished its exp2 pass of a tile
     uint32_t tmem_base;
     int abort_flag;
     int w[kMaxPairs];
@@ -266,8 +260,6 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
             mbar_init(&ctl->o_done[s], 1);
         }
         mbar_init(&ctl->drain, 2);  // one commit from each issuing warp
-        for (int t = 0; t < 2; ++t)
-            for (int q = 0; q < 4; ++q) mbar_init(&ctl->tok[t][q], 1);
         ctl->abort_flag = 0;
         fence_mbar_init();
     }
@@ -590,16 +582,6 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                 const float m_new = need ? tile_max : m_used;
                 const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
                 m_used = m_new;
-                // The two heads' warps on one SM sub-partition take turns at the exp2
-                // pass (head 0 of tile j, head 1 of tile j, head 0 of tile j+1, ...), so
-                // that the multi-function unit serves one of them at a time while the
-                // other loads S, corrects it and stores P.
-                if (F::Token && two) {
-                    wc.site = 14;
-                    if (t == 1) ok = mbar_wait_warp(&ctl->tok[0][q4], it & 1, wc);
-                    else if (it > 0) ok = mbar_wait_warp(&ctl->tok[1][q4], (it - 1) & 1, wc);
-                    if (!ok) break;
-                }
                 // P = exp2(s * scale - m) as bf16 pairs; S registers die as P is produced.
                 const float2 mneg = make_float2(-m_used, -m_used);
                 const float2 sc2 = make_float2(scale_log2, scale_log2);
@@ -609,26 +591,14 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                 for (int i = 0; i < 64; i += 2) {
                     float2 xa = fma2(make_float2(s[2 * i], s[2 * i + 1]), sc2, mneg);
                     float2 xb = fma2(make_float2(s[2 * i + 2], s[2 * i + 3]), sc2, mneg);
-                    if (((i) & 7) < kPolyPairsOf8) {
-                        xa = exp2_fma2(xa);
-                    } else {
-                        xa.x = fast_exp2(xa.x);
-                        xa.y = fast_exp2(xa.y);
-                    }
-                    if (((i + 1) & 7) < kPolyPairsOf8) {
-                        xb = exp2_fma2(xb);
-                    } else {
-                        xb.x = fast_exp2(xb.x);
-                        xb.y = fast_exp2(xb.y);
-                    }
+                    xa.x = fast_exp2(xa.x);
+                    xa.y = fast_exp2(xa.y);
+                    xb.x = fast_exp2(xb.x);
+                    xb.y = fast_exp2(xb.y);
                     l0 = add2(l0, xa);
                     l1 = add2(l1, xb);
                     pk[i] = pack_bf16x2(xa.x, xa.y);
                     pk[i + 1] = pack_bf16x2(xb.x, xb.y);
-                }
-                if (F::Token && two) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&ctl->tok[t][q4]);
                 }
                 // Rescale O only when some row's max grew past the threshold (rare).
                 // PV_t(j-1) must also be done reading P_t before it is overwritten.

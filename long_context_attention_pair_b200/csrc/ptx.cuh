@@ -273,28 +273,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     return d;
 }
 
-// exp2 of a pair on the FMA pipe.  Cody-Waite range reduction: n = round(x)
-// through the 1.5*2^23 magic add, f = x - n in [-1/2, 1/2]; 2^f by a degree-3
-// polynomial (weighted least-squares fit on Chebyshev nodes for relative error,
-// exact at f = 0; csrc/exp2_poly.py, max relative error 1.7e-4 in fp32); 2^n is
-// added to the exponent field: the integer n sits in the low mantissa bits of
-// x + 1.5*2^23, and shifting that word left by 23 leaves exactly n << 23.
-// Inputs are clamped to >= -125 (results below 2^-125 are far under bf16's
-// resolution of P; -inf maps to ~2^-125).
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-    x.x = fmaxf(x.x, -125.f);
-    x.y = fmaxf(x.y, -125.f);
-    const float2 magic = make_float2(12582912.f, 12582912.f);
-    const float2 t = add2(x, magic);
-    const float2 r = add2(t, make_float2(-12582912.f, -12582912.f));
-    const float2 f = fma2(r, make_float2(-1.f, -1.f), x);
-    float2 p = fma2(make_float2(0.055088684f, 0.055088684f), f, make_float2(0.24260405f, 0.24260405f));
-    p = fma2(p, f, make_float2(0.6932762f, 0.6932762f));
-    p = fma2(p, f, make_float2(1.f, 1.f));
-    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

@@ -6,6 +6,10 @@
 // into the device status word (first writer wins); the host maps any value at
 // or above the base to ATFLASH_ERR_TIMEOUT.
 #define ATFLASH_DEVICE_TIMEOUT_BASE 1000
+// A paged decode that met a page index past its block-table row, or a page id
+// outside the pool, writes this value (first writer wins); the host maps it to
+// ATFLASH_ERR_BAD_PAGE.
+#define ATFLASH_DEVICE_BAD_PAGE 2000
 
 // Waits that only let a CTA's own copies and tensor-core work finish before it
 // exits (after a pipeline wait has given up) use at least this limit, so that a

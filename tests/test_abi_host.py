@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for s in (0, -1, -2, -3, -4, -5, -6):
+    for s in (0, -1, -2, -3, -4, -5, -6, -7):
         assert atf.status_string(s) != "unknown status"
 
 
@@ -304,3 +304,27 @@ def test_theta_tables_rejected(L):
     assert L.atflash_theta_table(64, 1.0, (ctypes.c_double * 32)()) == -1
     with pytest.raises(ValueError):
         atf.window_table(64, 0.0, 1.0, 100, theta=good[:-1])
+
+
+def test_noalloc_decode_rejects_what_atflash_decode_rejects(L):
+    # The entry point that allocates nothing shares atflash_decode's argument
+    # checks: the same bad argument gives the same status (host only, nothing runs).
+    f = L.atflash_decode_noalloc
+    vp, i, i64, d = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+    f.argtypes = [vp, vp, vp, vp, vp, i, i, i, i64, i, d, d, i, i, i, i, vp]
+    f.restype = i
+    A, U = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8)  # never dereferenced
+    ws = ctypes.c_void_p(1 << 24)
+    good = dict(q=A, k=A, v=A, sl=A, out=A, B=2, Hq=8, Hkv=2, N=1000, D=128, base=1e4, kw=1.0, krot=0,
+                lay=atf.KV_HND, ind=atf.BF16, outd=atf.F32)
+    bad_cases = [dict(q=None), dict(B=0), dict(Hq=7), dict(N=0), dict(D=96), dict(D=65), dict(base=1.0),
+                 dict(kw=-1.0), dict(kw=float("nan")), dict(krot=2), dict(lay=7), dict(lay=atf.KV_PACKED),
+                 dict(lay=atf.KV_PACKED, krot=1, ind=atf.F32), dict(ind=5), dict(outd=5), dict(Hq=34, Hkv=2),
+                 dict(q=U), dict(out=U)]
+    for bad in bad_cases:
+        a = dict(good, **bad)
+        args = [a["q"], a["k"], a["v"], a["sl"], a["out"], a["B"], a["Hq"], a["Hkv"], a["N"], a["D"], a["base"],
+                a["kw"], a["krot"], a["lay"], a["ind"], a["outd"]]
+        rc_noalloc = f(*args, None)
+        rc_decode = L.atflash_decode(*args, ws, 1 << 30, None)
+        assert rc_noalloc < 0 and rc_noalloc == rc_decode, (bad, rc_noalloc, rc_decode)

@@ -133,8 +133,14 @@ def test_decode_qwen7b_1m_shape(oracle, kwin):
 
 
 @pytest.mark.slow
-def test_decode_qwen7b_128k_16_seqs(oracle):
-    decode_full_size(oracle, 16, 1 << 17, 16.0, seed=32)
+@pytest.mark.parametrize("kwin", [16.0, 64.0])
+def test_decode_qwen7b_128k_16_seqs(oracle, kwin):
+    decode_full_size(oracle, 16, 1 << 17, kwin, seed=32)
+
+
+@pytest.mark.slow
+def test_decode_qwen7b_128k_window_off(oracle):
+    decode_full_size(oracle, 16, 1 << 17, math.inf, seed=34)
 
 
 @pytest.mark.slow

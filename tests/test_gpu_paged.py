@@ -104,22 +104,28 @@ def test_paged_packed_equals_contiguous_packed(oracle, B, Hq, Hkv, L, D, P_, seq
     P.check(P.host(out), oref, "bf16", f"paged packed D={D}")
 
 
-def test_paged_bad_page_ids_read_zeros_without_fault():
-    B, Hq, Hkv, L, D, P_ = 1, 4, 2, 512, 128, 64
+@pytest.mark.parametrize("L,bad_index", [(512, 3), (512, 5), (100, 1)])
+def test_paged_bad_page_ids_are_reported(L, bad_index):
+    # A page id outside the pool or a negative one is an error the kernels find on
+    # the device: the status word reads ATFLASH_ERR_BAD_PAGE (no fault, no hang),
+    # and the next call with a valid table reads OK again.  L = 100 takes the
+    # short-sequence fp32 path too.
+    B, Hq, Hkv, D, P_ = 1, 4, 2, 128, 64
     q = P.gen(75, "q_dec", (B, Hq, D), "bf16")
-    kc = P.gen(75, "k_cache", (B, Hkv, L, D), "bf16")
-    vc = P.gen(75, "v_cache", (B, Hkv, L, D), "bf16")
-    ids, n_pool = scatter_pages(B, Hkv, L, P_, 76)
+    kc = P.gen(75, "k_cache", (B, Hkv, 512, D), "bf16")
+    vc = P.gen(75, "v_cache", (B, Hkv, 512, D), "bf16")
+    ids, n_pool = scatter_pages(B, Hkv, 512, P_, 76)
     kp, vp = nhd_pool(kc, ids, n_pool, P_), nhd_pool(vc, ids, n_pool, P_)
-    bad = ids.copy()
-    bad[0, 3] = 10 ** 7   # outside the pool
-    bad[0, 5] = -4
     sl = torch.tensor([L], dtype=torch.int32, device="cuda")
-    out = atf.decode_paged(q, kp, vp, torch.as_tensor(bad, device="cuda"), sl, P_, 1e7, 16.0,
-                           out_dtype=torch.float32)
+    assert atf.device_status() == 0
+    bad = ids.copy()
+    bad[0, bad_index] = 10 ** 7 if bad_index != 5 else -4
+    atf.decode_paged(q, kp, vp, torch.as_tensor(bad, device="cuda"), sl, P_, 1e7, 16.0, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert atf.device_status() == atf.ERR_BAD_PAGE
+    atf.decode_paged(q, kp, vp, torch.as_tensor(ids, device="cuda"), sl, P_, 1e7, 16.0, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert atf.device_status() == 0
-    assert torch.isfinite(out).all()
 
 
 @pytest.mark.slow

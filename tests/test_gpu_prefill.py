@@ -143,12 +143,24 @@ def test_qwen05b_shape_32k(oracle):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("N", [8192, 131072])
+@pytest.mark.parametrize("N", [8192, 32768, 131072])
 def test_llama3b_shape(oracle, N):
     sampled_parity(oracle, 1, N, 24, 8, 128, 5e5, 16.0, seed=12)
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("N,kwin", [(262144, 16.0), (524288, 64.0)])
+@pytest.mark.parametrize("N,kwin", [(262144, 16.0), (262144, 64.0), (524288, 16.0), (524288, 64.0)])
 def test_qwen7b_1m_shape(oracle, N, kwin):
     sampled_parity(oracle, 1, N, 28, 4, 128, 1e7, kwin, seed=13)
+
+
+# Window off (k = inf) at workload size: the one-head D = 64 form (two CTAs per SM)
+# and the two-head D = 128 form over every key tile.
+@pytest.mark.slow
+def test_qwen05b_shape_32k_window_off(oracle):
+    sampled_parity(oracle, 1, 32768, 14, 2, 64, 1e6, math.inf, seed=14)
+
+
+@pytest.mark.slow
+def test_llama3b_shape_128k_window_off(oracle):
+    sampled_parity(oracle, 1, 131072, 24, 8, 128, 5e5, math.inf, seed=15)

@@ -40,8 +40,9 @@ def test_scaled_prefill_matches_oracle(oracle, B, N, Hq, Hkv, D, base, kwin, dty
 
 @pytest.mark.parametrize("D,base,kwin", [(64, 1e6, 8.0), (128, 5e5, 16.0)])
 def test_scaled_packed_prefill_equals_scaled_prefill(D, base, kwin):
-    # rope_pack + prefill_packed with a scaled table is the same computation as the
-    # one-call prefill with that table (which carves the same packed scratch).
+    # rope_pack + prefill_packed + prefill_short_rows with a scaled table is the
+    # same computation as the one-call prefill with that table (which carves the
+    # same packed scratch and runs the same three steps).
     th = llama3_scaled_theta(D, base, factor=32.0, orig_ctx=512.0)
     q = P.gen(74, "q", (1, 2000, 6, D), "bf16")
     k = P.gen(74, "k", (1, 2000, 2, D), "bf16")
@@ -49,12 +50,14 @@ def test_scaled_packed_prefill_equals_scaled_prefill(D, base, kwin):
     qp = atf.rope_pack(q, 0.0, theta=th)
     kp = atf.rope_pack(k, 0.0, theta=th)
     a = atf.prefill_packed(qp, kp, v, 0.0, kwin, theta=th)
+    atf.prefill_short_rows(q, k, v, a, 0.0, kwin, theta=th)
     b = atf.prefill(q, k, v, 0.0, kwin, theta=th)
     torch.cuda.synchronize()
     assert atf.device_status() == 0
     assert torch.equal(a, b)
     # and not what the unscaled base table gives
     c = atf.prefill_packed(atf.rope_pack(q, base), atf.rope_pack(k, base), v, base, kwin)
+    atf.prefill_short_rows(q, k, v, c, base, kwin)
     torch.cuda.synchronize()
     assert not torch.equal(a, c)
 
