@@ -54,8 +54,10 @@ constexpr float kRescaleThreshold = 8.0f;
 
 template <int D>
 struct Cfg {
-    // Two stages per CTA and three CTAs per SM (74 KB of shared memory each): more
-    // consumer warps to hide latency, as many bytes in flight as three stages at two.
+    // Two stages per CTA and three CTAs per SM (69 KB of dynamic shared memory each,
+    // plus at most 3 KB of static tables and the 1 KB the hardware reserves per CTA):
+    // more consumer warps to hide latency, as many bytes in flight as three stages at
+    // two.  The rotated queries are kept as bf16 (the MMA operand) so that three fit.
     static constexpr int kStages = 2;
     static constexpr int H = D / 2;
     static constexpr int C = D / 16;                   // chunks of 8 pairs
@@ -66,10 +68,11 @@ struct Cfg {
     static constexpr int OffK = 0;
     static constexpr int OffV = OffK + kStages * KBytes;
     static constexpr int OffBase = OffV + kStages * VBytes;      // [stage][H] float
-    static constexpr int OffQ = OffBase + kStages * H * 4;       // [16][D] float, rotated queries
-    static constexpr int OffBar = OffQ + 16 * D * 4;
+    static constexpr int OffQ = OffBase + kStages * H * 4;       // [16][D] bf16, rotated queries
+    static constexpr int OffBar = OffQ + 16 * D * 2;
     static constexpr int Total = OffBar + 256;
     static constexpr int Request = Total + 1024;
+    static_assert(3 * (Request + 3072 + 1024) <= 233472, "three CTAs must fit the SM's 228 KB");
 };
 
 constexpr int kMaxStages = 8;
@@ -110,6 +113,11 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Two bf16 values as one register (lo in the low half).
+__device__ __forceinline__ uint32_t bf16_pair(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+    return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+}
+
 // Rotate the two pairs held in (lo, hi) = (dims r|r+1 of the low half, dims
 // r+H|r+1+H) of one key, and zero a pair whose window the key exceeds.
 __device__ __forceinline__ void rotate_pairs(uint32_t &lo, uint32_t &hi, float c0, float s0, float c1, float s1,
@@ -148,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
     uint8_t *sK = smem + F::OffK;
     uint8_t *sV = smem + F::OffV;
     float *sBase = reinterpret_cast<float *>(smem + F::OffBase);
-    float *sQ = reinterpret_cast<float *>(smem + F::OffQ);
+    __nv_bfloat16 *sQ = reinterpret_cast<__nv_bfloat16 *>(smem + F::OffQ);
     Bars *bars = reinterpret_cast<Bars *>(smem + F::OffBar);
     __shared__ int sw[kMaxPairs];
     __shared__ float sTheta[kMaxPairs];
@@ -197,8 +205,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
             xr = a * cs - c * sn;
             xh = c * cs + a * sn;
         }
-        sQ[j * D + r] = xr;
-        sQ[j * D + r + H] = xh;
+        // Rounded once to bf16 here: the MMA's B operand.
+        sQ[j * D + r] = __float2bfloat16_rn(xr);
+        sQ[j * D + r + H] = __float2bfloat16_rn(xh);
     }
     __syncthreads();
     WaitCtl wc{&bars->abort_flag, status, limit_ns, 20};
@@ -314,17 +323,17 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
         for (int c = 0; c < C; ++c) {
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-                const float *qrow = sQ + (8 * t + gq) * D;
+                const __nv_bfloat16 *qrow = sQ + (8 * t + gq) * D;
                 if (kPacked) {
                     // k-order of a packed chunk: (pair 8c + k/2, component k%2).
                     const int pa = 8 * c + tq, pb = pa + 4;
-                    qb[c][t][0] = pack_bf16x2(qrow[pa], qrow[pa + H]);
-                    qb[c][t][1] = pack_bf16x2(qrow[pb], qrow[pb + H]);
+                    qb[c][t][0] = bf16_pair(qrow[pa], qrow[pa + H]);
+                    qb[c][t][1] = bf16_pair(qrow[pb], qrow[pb + H]);
                 } else {
-                    // k-order [dims 8c..8c+7, dims H+8c..H+8c+7].
+                    // k-order [dims 8c..8c+7, dims H+8c..H+8c+7]: two adjacent bf16 per register.
                     const int lo = 8 * c + 2 * tq, hi = H + 8 * c + 2 * tq;
-                    qb[c][t][0] = pack_bf16x2(qrow[lo], qrow[lo + 1]);
-                    qb[c][t][1] = pack_bf16x2(qrow[hi], qrow[hi + 1]);
+                    qb[c][t][0] = *reinterpret_cast<const uint32_t *>(qrow + lo);
+                    qb[c][t][1] = *reinterpret_cast<const uint32_t *>(qrow + hi);
                 }
             }
         }
@@ -695,6 +704,9 @@ cudaError_t launch_decode_tc(const void *q, const void *kc, const void *vc, cons
         const int smem = dtc::Cfg<DD>::Request;                                                                \
         if ((e = cudaFuncSetAttribute(dtc::decode_tc_kernel<DD, PK, PG, NT>,                                  \
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)      \
+            return e;                                                                                          \
+        if ((e = cudaFuncSetAttribute(dtc::decode_tc_kernel<DD, PK, PG, NT>,                                  \
+                                      cudaFuncAttributePreferredSharedMemoryCarveout, 100)) != cudaSuccess)    \
             return e;                                                                                          \
         dtc::decode_tc_kernel<DD, PK, PG, NT><<<grid, dtc::kThreads, smem, s>>>(                              \
             tk, tv, q, seqlens, workspace, p.Hq, p.Hkv, nhd, krot, split_keys, nsplit, wp, status, limit_ns,  \
