@@ -289,15 +289,20 @@ KERNELS_PER_STEP = 7
 # DRAM bytes per launch of the tcgen05 prefill kernel, from one ncu capture per
 # workload.  Valid only while the kernel source hashes to `source_sha1`;
 # otherwise the line reports null.
-TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98168320,
-           "source_sha1": "fd039e524fa9ed078dfba5e3b08f3de1cb0a5392"}
-# DRAM bytes per launch of the decode kernel (split states included, merge not) on
-# the full-size workloads, from ncu captures; valid while decode_tc.cu hashes to
-# `source_sha1`.
-DECODE_TRAFFIC = {"decode_1m_packed": {"bytes_per_launch": 6607293952,
-                                       "source_sha1": "61a5dcf9b9fce74f5022cf838de7d70f2150435d"},
-                  "decode_1m": {"bytes_per_launch": 8608907008,
-                                "source_sha1": "61a5dcf9b9fce74f5022cf838de7d70f2150435d"}}
+TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98121216,
+           "source_sha1": "547e2804942e61a0beac9f41647b250d25b3670d"}
+# DRAM bytes per launch of the decode kernel (split states included, merge not),
+# from an ncu capture of the same workload at a shorter cache length
+# `captured_L`; valid while decode_tc.cu hashes to `source_sha1`.  The natural
+# layouts read the whole cache whatever the window (every 128-byte half-row keeps
+# a sector), so their traffic grows in proportion to L and is scaled to the
+# line's L; the packed layout's kept share depends on L, so it is reported only
+# at the captured length.
+DECODE_TRAFFIC = {"decode_1m": {"captured_L": 131072, "bytes_per_launch": 1078800128, "proportional_to_L": True,
+                                "source_sha1": "3f0aa78370ba9c79bdc31255877b0817885b25c3"},
+                  "decode_1m_packed": {"captured_L": 131072, "bytes_per_launch": 897253632,
+                                       "proportional_to_L": False,
+                                       "source_sha1": "3f0aa78370ba9c79bdc31255877b0817885b25c3"}}
 
 
 def parse():
@@ -345,11 +350,15 @@ def prefill_traffic(workload, wl):
 
 
 def decode_traffic(workload, L):
-    """Captured DRAM bytes of one decode launch for this workload, or None."""
+    """Captured DRAM bytes of one decode launch for this workload at cache length L, or None."""
     rec = DECODE_TRAFFIC.get(workload)
-    if rec is None or L != DECODE_WORKLOADS[workload]["N"] or rec["source_sha1"] != kernel_sha1("decode_tc.cu"):
+    if rec is None or rec["source_sha1"] != kernel_sha1("decode_tc.cu"):
         return None
-    return rec["bytes_per_launch"]
+    if L == rec["captured_L"]:
+        return rec["bytes_per_launch"]
+    if rec.get("proportional_to_L"):
+        return round(rec["bytes_per_launch"] * L / rec["captured_L"])
+    return None
 
 
 def dist_setup():
