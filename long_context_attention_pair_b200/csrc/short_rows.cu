@@ -129,9 +129,9 @@ __device__ __forceinline__ float2 sr_key_pair(const Src &s, int b, int kvh, int6
 }
 
 // kDecode = false: grid (candidate query tiles, work items, B*Hkv); a work item is
-// (32-row slice, query head of the group); dense and ragged launches take one item
-// per CTA (gridDim.y = 4G) and only query tile 0, block-selected launches every
-// query tile with the items looped in the CTA (gridDim.y = 1).
+// (32-row slice, query head of the group), one per CTA (gridDim.y = 4G).  Dense and
+// ragged launches take only query tile 0; block-selected launches every query tile,
+// and a CTA whose tile keeps an earlier key tile exits after scanning the mask row.
 // kDecode = true: grid (1, 1, B*Hkv); the rows are the group's query heads.
 template <int D, bool kDecode>
 __global__ void __launch_bounds__(kThreads) short_rows_kernel(const __grid_constant__ Args a,
@@ -373,7 +373,7 @@ cudaError_t launch_short_rows_prefill(const void *q, const void *k, const void *
     a.num_qt = (int)((p.N + sr::kTile - 1) / sr::kTile);
     a.status = status;
     const unsigned z = (unsigned)(p.B * p.Hkv);
-    const dim3 grid = block_mask ? dim3((unsigned)a.num_qt, 1, z) : dim3(1, (unsigned)(4 * a.G), z);
+    const dim3 grid((unsigned)(block_mask ? a.num_qt : 1), (unsigned)(4 * a.G), z);
     if (p.D == 128) return sr::launch<128, false>(a, wp, grid, s);
     if (p.D == 64) return sr::launch<64, false>(a, wp, grid, s);
     return cudaErrorInvalidValue;
