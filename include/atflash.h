@@ -197,7 +197,10 @@ size_t atflash_rope_pack_bytes(int B, int64_t N, int H, int D, int in_dtype);
 /*
  * Windowed attention over already rotated, packed queries and keys (outputs of
  * atflash_rope_pack with the same in_dtype, B, N, D and rope_base).  Same
- * semantics, layouts of v/out/lse and constraints as atflash_prefill_ex.
+ * semantics, layouts of v/out/lse and constraints as atflash_prefill_ex, except
+ * that the short-row step (see "Accuracy of short rows") is not part of this
+ * call: it needs the un-rotated inputs, so queue atflash_prefill_short_rows
+ * after it on the same stream to get atflash_prefill_ex's bits (bf16).
  */
 int atflash_prefill_packed(const void *qpack, const void *kpack, const void *v, void *out, int B, int Hq,
                            int Hkv, int64_t N, int D, double rope_base, double k_window, int in_dtype,
