@@ -461,7 +461,7 @@ class ClockSampler:
 def oracle_rows_per_step(wl):
     """Query rows (all heads) the oracle computes per step, one rule for both arms:
     about 2^33 / (N * Hq * D) rows, so that a step is about a second of host work
-    whatever the workload (5 rows at the 512K default, 292 at 32K)."""
+    whatever the workload (5 rows at the 512K default, 293 at 32K)."""
     return max(1, round(2 ** 33 / (wl["N"] * wl["Hq"] * wl["D"])))
 
 

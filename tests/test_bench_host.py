@@ -91,3 +91,21 @@ def test_block_mask_recipe_shape_and_structure():
     assert np.all(np.diag(m[0, 0]) == 1)                         # local band includes the diagonal
     assert np.all(m[0, :, wl["sink_tiles"]:, :wl["sink_tiles"]] == 1)
     assert np.array_equal(m, bench.block_mask_recipe(wl, T))    # seeded
+
+
+def test_default_line_is_the_largest_single_gpu_prefill_config():
+    wl = bench.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    assert (wl["N"], wl["Hq"], wl["Hkv"], wl["D"], wl["k_window"]) == (524288, 28, 4, 128, 16.0)
+    assert max(w["N"] for w in bench.WORKLOADS.values()) == wl["N"]
+    for name in bench.SUB_RECORDS:
+        assert name in bench.WORKLOADS or name in bench.DECODE_WORKLOADS
+
+
+def test_both_arms_sample_the_oracle_by_one_rule_and_report_one_config():
+    assert bench.oracle_rows_per_step(bench.WORKLOADS["qwen7b_512k"]) == 5
+    assert bench.oracle_rows_per_step(bench.WORKLOADS["qwen05b_32k"]) == 293
+    for wl in bench.WORKLOADS.values():
+        assert bench.oracle_rows_per_step(wl) >= 1
+        for world in (1, 2, 8):
+            assert bench.line_config(dict(wl), world) == bench.line_config(dict(wl), world)
+            assert bench.line_config(dict(wl), world)["parallelism"] == ("replicas" if world > 1 else "single GPU")

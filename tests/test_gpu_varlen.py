@@ -106,3 +106,21 @@ def test_varlen_bench_mix_sampled(oracle, name, rows):
     torch.cuda.synchronize()
     assert atf.device_status() == 0
     check_against_oracle(oracle, q, k, v, cu, out, wl["rope_base"], wl["k_window"], max_rows=rows, seed=65)
+
+
+def test_varlen_first_tile_rows_are_exact(oracle):
+    # Rows 0..127 of every sequence see at most 128 keys and are computed in fp32.
+    lens, Hq, Hkv, D, base, kwin = [1, 77, 128, 129, 300], 6, 2, 128, 5e5, 16.0
+    q, k, v, cu = packed_batch(66, lens, Hq, Hkv, D)
+    out, lse = atf.prefill_varlen(q, k, v, torch.as_tensor(cu, device="cuda"), max(lens), base, kwin,
+                                  out_dtype=torch.float32, return_lse=True)
+    torch.cuda.synchronize()
+    assert atf.device_status() == 0
+    for b in range(len(lens)):
+        t0, n = int(cu[b]), lens[b]
+        rows = np.arange(min(n, 128))
+        idx = torch.as_tensor(t0 + rows, device="cuda")
+        ref, rlse = oracle.prefill_rows(P.host(q[idx]), rows, P.host(k[t0:t0 + n]), P.host(v[t0:t0 + n]), base,
+                                        kwin, want_lse=True)
+        P.check(P.host(out[idx]), ref, "f32", f"varlen seq {b} first tile")
+        P.check(P.host(lse[:, idx]).T, rlse, "f32", f"varlen seq {b} first-tile lse")
