@@ -328,3 +328,18 @@ def test_noalloc_decode_rejects_what_atflash_decode_rejects(L):
         rc_noalloc = f(*args, None)
         rc_decode = L.atflash_decode(*args, ws, 1 << 30, None)
         assert rc_noalloc < 0 and rc_noalloc == rc_decode, (bad, rc_noalloc, rc_decode)
+
+
+def test_short_rows_step_argument_errors(L):
+    # The short-row step on its own rejects what atflash_prefill_ex rejects for bf16 input.
+    A, U = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8)
+    f = L.atflash_prefill_short_rows
+    assert f(None, A, A, A, 1, 2, 1, 256, 64, 1e4, 1.0, atf.BF16, None, None) == -1
+    assert f(A, A, A, A, 1, 3, 2, 256, 64, 1e4, 1.0, atf.BF16, None, None) == -1      # Hq % Hkv
+    assert f(A, A, A, A, 1, 2, 1, 256, 64, 1.0, 1.0, atf.BF16, None, None) == -1      # base <= 1
+    assert f(A, A, A, A, 1, 2, 1, 256, 64, 1e4, -1.0, atf.BF16, None, None) == -1     # k < 0
+    assert f(A, A, A, A, 1, 2, 1, 256, 96, 1e4, 1.0, atf.BF16, None, None) == -2      # D
+    assert f(A, A, A, A, 1, 2, 1, 256, 64, 1e4, 1.0, 7, None, None) == -2             # out dtype
+    assert f(U, A, A, A, 1, 2, 1, 256, 64, 1e4, 1.0, atf.BF16, None, None) == -6      # alignment
+    g = L.atflash_prefill_short_rows_theta
+    assert g(A, A, A, A, 1, 2, 1, 256, 64, None, 1.0, atf.BF16, None, None) == -1     # no table
