@@ -476,21 +476,16 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                 if (!(ok = mbar_wait_warp(&ctl->s_full[t], it & 1, wc))) break;
                 tc_fence_after();
                 if ((bd.r_lo >> 3) < C) {
-                    uint32_t r0[32], r1[32], r2[32], r3[32];
-                    tmem_ld_32x32b_x32(tS + 0, r0);
-                    tmem_ld_32x32b_x32(tS + 32, r1);
-                    tmem_ld_32x32b_x32(tS + 64, r2);
-                    tmem_ld_32x32b_x32(tS + 96, r3);
-                    tmem_ld_wait(r0);
-                    tmem_ld_wait(r1);
-                    tmem_ld_wait(r2);
-                    tmem_ld_wait(r3);
+                    // Two 64-column loads (measured faster than four of 32 columns at D = 128).
+                    uint32_t ra[64], rb[64];
+                    tmem_ld_32x32b_x64(tS + 0, ra);
+                    tmem_ld_32x32b_x64(tS + 64, rb);
+                    tmem_ld_wait(ra);
+                    tmem_ld_wait(rb);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        s[i] = __uint_as_float(r0[i]);
-                        s[32 + i] = __uint_as_float(r1[i]);
-                        s[64 + i] = __uint_as_float(r2[i]);
-                        s[96 + i] = __uint_as_float(r3[i]);
+                    for (int i = 0; i < 64; ++i) {
+                        s[i] = __uint_as_float(ra[i]);
+                        s[64 + i] = __uint_as_float(rb[i]);
                     }
                 } else {
 #pragma unroll
