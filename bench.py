@@ -289,8 +289,8 @@ KERNELS_PER_STEP = 7
 # DRAM bytes per launch of the tcgen05 prefill kernel, from one ncu capture per
 # workload.  Valid only while the kernel source hashes to `source_sha1`;
 # otherwise the line reports null.
-TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98121216,
-           "source_sha1": "547e2804942e61a0beac9f41647b250d25b3670d"}
+TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98064384,
+           "source_sha1": "f7beae16cba2cfe4917e7b8359504532336667e3"}
 # DRAM bytes per launch of the decode kernel (split states included, merge not),
 # from an ncu capture of the same workload at a shorter cache length
 # `captured_L`; valid while decode_tc.cu hashes to `source_sha1`.  The natural
