@@ -289,8 +289,8 @@ KERNELS_PER_STEP = 7
 # DRAM bytes per launch of the tcgen05 prefill kernel, from one ncu capture per
 # workload.  Valid only while the kernel source hashes to `source_sha1`;
 # otherwise the line reports null.
-TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98064384,
-           "source_sha1": "f7beae16cba2cfe4917e7b8359504532336667e3"}
+TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98543616,
+           "source_sha1": "0d19d32cb15f5f9de5107841ea5bf3503b043c96"}
 # DRAM bytes per launch of the decode kernel (split states included, merge not),
 # from an ncu capture of the same workload at a shorter cache length
 # `captured_L`; valid while decode_tc.cu hashes to `source_sha1`.  The natural

@@ -476,16 +476,26 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                 if (!(ok = mbar_wait_warp(&ctl->s_full[t], it & 1, wc))) break;
                 tc_fence_after();
                 if ((bd.r_lo >> 3) < C) {
-                    // Two 64-column loads (measured faster than four of 32 columns at D = 128).
-                    uint32_t ra[64], rb[64];
-                    tmem_ld_32x32b_x64(tS + 0, ra);
-                    tmem_ld_32x32b_x64(tS + 64, rb);
-                    tmem_ld_wait(ra);
-                    tmem_ld_wait(rb);
+                    // The whole row in one 128-column load in the two-head kernel, two 64-column
+                    // loads in the one-head kernel (128 registers at launch); both measured faster
+                    // than four loads of 32 columns.
+                    if constexpr (NH == 2) {
+                        uint32_t ra[128];
+                        tmem_ld_32x32b_x128(tS, ra);
+                        tmem_ld_wait(ra);
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        s[i] = __uint_as_float(ra[i]);
-                        s[64 + i] = __uint_as_float(rb[i]);
+                        for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(ra[i]);
+                    } else {
+                        uint32_t ra[64], rb[64];
+                        tmem_ld_32x32b_x64(tS + 0, ra);
+                        tmem_ld_32x32b_x64(tS + 64, rb);
+                        tmem_ld_wait(ra);
+                        tmem_ld_wait(rb);
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) {
+                            s[i] = __uint_as_float(ra[i]);
+                            s[64 + i] = __uint_as_float(rb[i]);
+                        }
                     }
                 } else {
 #pragma unroll
@@ -552,8 +562,8 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                             }
                         }
                     }
+                    __syncwarp();  // every lane is done with this stage's staged keys
                 }
-                __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->k_empty[ks]);
                 // Causal mask on the diagonal tile; row max of the raw scores (4 chains
                 // of 3-input max); the 1/sqrt(D) * log2(e) scale is folded into the exp.
