@@ -293,11 +293,12 @@ TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98543616,
            "source_sha1": "0d19d32cb15f5f9de5107841ea5bf3503b043c96"}
 # DRAM bytes per launch of the decode kernel (split states included, merge not),
 # from an ncu capture of the same workload at a shorter cache length
-# `captured_L`; valid while decode_tc.cu hashes to `source_sha1`.  The natural
+# `captured_L`; valid while decode_tc.cu and decode.cu (the split heuristic)
+# hash to `source_sha1`.  The natural
 # layouts read the whole cache whatever the window (every 128-byte half-row keeps
-# a sector), so their traffic grows in proportion to L and is scaled to the
-# line's L; the packed layout's kept share depends on L, so it is reported only
-# at the captured length.
+# a sector), so their traffic grows in proportion to B * L and is scaled to the
+# line's; the packed layout's kept share depends on L, so it is reported only at
+# the captured length and the workload's own B.
 DECODE_TRAFFIC = {"decode_1m": {"captured_L": 131072, "bytes_per_launch": 1078800128, "proportional_to_L": True,
                                 "source_sha1": "3f0aa78370ba9c79bdc31255877b0817885b25c3"},
                   "decode_1m_packed": {"captured_L": 131072, "bytes_per_launch": 897253632,
@@ -318,6 +319,7 @@ def parse():
                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(VARLEN_WORKLOADS) +
                    sorted(SPARSE_WORKLOADS))
     p.add_argument("--N", type=int, default=None, help="override sequence length (sweeps)")
+    p.add_argument("--B", type=int, default=None, help="override the number of sequences (decode sweeps)")
     p.add_argument("--k-window", type=float, default=None, help="override k (inf = window off)")
     return p.parse_args()
 
@@ -331,10 +333,17 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_sha1(name="prefill_tc.cu"):
-    path = os.path.join(ROOT, "long_context_attention_pair_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha1(f.read()).hexdigest()
+def kernel_sha1(*names):
+    """sha1 of the named kernel sources, concatenated (default: the prefill kernel's)."""
+    h = hashlib.sha1()
+    for name in names or ("prefill_tc.cu",):
+        with open(os.path.join(ROOT, "long_context_attention_pair_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+# The decode kernel and the split heuristic that sets its launch (keys per CTA).
+DECODE_SOURCES = ("decode_tc.cu", "decode.cu")
 
 
 # ---------------------------------------------------------------- distributed
@@ -349,15 +358,18 @@ def prefill_traffic(workload, wl):
     return TRAFFIC["bytes_per_launch"]
 
 
-def decode_traffic(workload, L):
-    """Captured DRAM bytes of one decode launch for this workload at cache length L, or None."""
+def decode_traffic(workload, L, B=None):
+    """Captured DRAM bytes of one decode launch for this workload at cache length L
+    (and B sequences, default the workload's), or None."""
     rec = DECODE_TRAFFIC.get(workload)
-    if rec is None or rec["source_sha1"] != kernel_sha1("decode_tc.cu"):
+    if rec is None or rec["source_sha1"] != kernel_sha1(*DECODE_SOURCES):
         return None
-    if L == rec["captured_L"]:
+    B0 = DECODE_WORKLOADS[workload]["B"]
+    B = B0 if B is None else B
+    if L == rec["captured_L"] and B == B0:
         return rec["bytes_per_launch"]
     if rec.get("proportional_to_L"):
-        return round(rec["bytes_per_launch"] * L / rec["captured_L"])
+        return round(rec["bytes_per_launch"] * (B * L) / (B0 * rec["captured_L"]))
     return None
 
 
@@ -780,10 +792,26 @@ def measure_decode(args, wl, name, dev):
         def call(kw):
             atf.decode(q, kc, vc, sl, base, kw, out=out, workspace=ws, **dkw)
 
+    cache_bytes = 2 * B * Hkv * L * D * 2
+    # A cache that L2 could hold is evicted before every call (a 256 MiB write
+    # outside the timed events), so that each call reads it from HBM as a decode
+    # step of a many-layer model would; larger caches stream back to back.
+    small = cache_bytes < 2 * L2_FLUSH_BYTES
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if small else None
+
     def timed(kw, steps):
         for _ in range(args.warmup):
             call(kw)
         torch.cuda.synchronize()
+        if small:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for a, b in evs:
+                flush.zero_()
+                a.record(stream)
+                call(kw)
+                b.record(stream)
+            torch.cuda.synchronize()
+            return sum(a.elapsed_time(b) for a, b in evs) / steps
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(steps):
@@ -808,10 +836,12 @@ def measure_decode(args, wl, name, dev):
     line = {"metric": METRIC, "value": round(world * B / (ms / 1e3), 2), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(wl, l2="inputs larger than L2 (cache of %.1f GB)" % (2 * B * Hkv * L * D * 2 / 1e9)),
+            "config": dict(wl, l2=("L2 flushed before every call (256 MiB write, outside the timed events; cache of "
+                                   "%.1f MB)" % (cache_bytes / 1e6)) if small else
+                           "inputs larger than L2 (cache of %.1f GB)" % (cache_bytes / 1e9)),
             "decode": {"us_per_call": round(1e3 * ms, 2), "us_per_token": round(1e3 * ms / B, 2)},
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": decode_traffic(name, L),
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": decode_traffic(name, L, B),
                          "kernel": f"decode_tc_kernel<{D}{', paged' if page else ''}> + decode_merge_kernel",
                          "bytes_per_call": nbytes, "peak_source": src},
             "window_off": {"ms_per_step": round(ms_off, 4), "us_per_token": round(1e3 * ms_off / B, 2)},
@@ -1050,6 +1080,8 @@ def main():
         wl = dict(DECODE_WORKLOADS[args.workload])
         if args.N:
             wl["N"] = args.N
+        if args.B:
+            wl["B"] = args.B
         if args.k_window is not None:
             wl["k_window"] = args.k_window
         run_decode(args, wl)

@@ -21,15 +21,21 @@ namespace atf {
 constexpr int kDecodeWarps = 4;
 constexpr int kMaxGroup = 16;  // query heads per KV head
 
-// Keys per split: enough (sequence, KV head, split) CTAs to fill 148 SMs twice,
-// a multiple of 256 keys, at most 4096.
+// Keys per split: a multiple of 64 (one TMA stage of the tensor-core kernel)
+// between 256 and 4096, chosen so that the (sequence, KV head, split) CTAs come
+// close to, without passing, a whole number of waves of that kernel's 148 SMs x
+// 3 resident CTAs: a last wave that is mostly empty streams at a fraction of
+// the HBM bandwidth.
 int decode_split_keys(int B, int Hkv, int64_t Nmax) {
-    const int64_t total = (int64_t)B * Hkv * Nmax;
-    int64_t per = (total + 295) / 296;
-    per = (per + 255) / 256 * 256;
-    if (per < 256) per = 256;
-    if (per > 4096) per = 4096;
-    return (int)per;
+    constexpr int64_t kSlots = 148 * 3, kUnit = 64, kMinUnits = 4, kMaxUnits = 64;
+    const int64_t units = (Nmax + kUnit - 1) / kUnit;  // stages per (sequence, KV head)
+    const int64_t pairs = (int64_t)B * Hkv;
+    const int64_t waves = (pairs * units + kSlots * kMaxUnits - 1) / (kSlots * kMaxUnits);
+    int64_t splits = waves * kSlots / pairs;  // per (sequence, KV head)
+    if (splits < 1) splits = 1;
+    int64_t per = (units + splits - 1) / splits;
+    per = per < kMinUnits ? kMinUnits : (per > kMaxUnits ? kMaxUnits : per);
+    return (int)(per * kUnit);
 }
 
 int decode_num_splits(int B, int Hkv, int64_t Nmax) {
@@ -213,6 +219,9 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float
                                                                      int out_f32, int Hq, int nsplit, int D) {
     __shared__ float red[32];
     __shared__ float part_acc[kMergeParts][kMergeDims];
+    // Launched as a dependent of the split kernel: wait for its states.
+    pdl_wait();
+    pdl_allow_dependents();
     const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     const float *base = ws + ((size_t)b * Hq + h) * nsplit * (D + 2);
     float mx = -INFINITY;
@@ -278,9 +287,11 @@ cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const i
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<<<dim3((unsigned)p.Hq, (unsigned)p.B, (unsigned)(p.D / kMergeDims)), kMergeThreads, 0, s>>>(
-        workspace, out, out_f32, p.Hq, nsplit, p.D);
-    if ((e = cudaGetLastError()) != cudaSuccess || in_f32) return e;
+    // The merge and the short decode rows are launched as programmatic dependents,
+    // so that their launch overlaps the tail of the kernel before them.
+    e = launch_dependent(decode_merge_kernel, dim3((unsigned)p.Hq, (unsigned)p.B, (unsigned)(p.D / kMergeDims)),
+                         dim3(kMergeThreads), 0, s, (const float *)workspace, out, out_f32, p.Hq, nsplit, p.D);
+    if (e != cudaSuccess || in_f32) return e;
     // bf16 caches: sequences of at most 128 tokens again in fp32 (the fp32 path is exact already).
     int *status = device_status_word();
     if (!status) return cudaErrorUnknown;

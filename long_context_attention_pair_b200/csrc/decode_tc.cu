@@ -87,6 +87,17 @@ __device__ __forceinline__ int walk_down(const int *w, int r, int d) {
     while (r > 0 && w[r - 1] >= d) --r;
     return r;
 }
+// The walks' starting points: r*(d) = the smallest r with w_r >= d (H when none),
+// by bisection (the windows do not decrease in r).  Walking down from H instead
+// took up to H dependent shared-memory reads before a CTA's first stage.
+__device__ __forceinline__ int first_kept_pair(const int *w, int H, int d) {
+    int lo = 0, hi = H;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (w[mid] >= d) hi = mid; else lo = mid + 1;
+    }
+    return lo;
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &d0, uint32_t &d1, uint32_t &d2, uint32_t &d3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -210,6 +221,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
         sQ[j * D + r + H] = __float2bfloat16_rn(xh);
     }
     __syncthreads();
+    pdl_allow_dependents();  // the merge may be scheduled now; it waits for this grid to complete
     WaitCtl wc{&bars->abort_flag, status, limit_ns, 20};
 
     if (warp == kConsumers) {
@@ -225,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
         const bool rotate = !kPacked && !krot;
         // r*(d) of the stage's nearest key: stages move towards the query, so the
         // first kept pair only moves down (amortised O(1) per stage).
-        int r_near = H;
+        int r_near = first_kept_pair(sw, H, (int)((L - 1) - (s0 + kStageKeys - 1 < s1 ? s0 + kStageKeys - 1 : s1 - 1)));
         for (int it = 0; it < nstage && ok; ++it) {
             const int st = it % kStages;
             const int64_t k0 = s0 + (int64_t)it * kStageKeys;
@@ -354,8 +366,15 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 1) decode_tc_kernel(
         // Positions fit in int32 (Nmax <= 2^31 - 1).  Walk pointers for r*(d) of the
         // stage's nearest key, this warp's nearest key and this warp's farthest key.
         const int Lq = (int)L - 1;
-        int r_stage = H, r_warp = H, r_keep = H;
         const int grp = warp / kWarpsPerStage, wq = warp % kWarpsPerStage;
+        int r_stage = H, r_warp = H, r_keep = H;
+        if (grp < nstage) {
+            // Start the walks at this warp's first stage.
+            const int k0 = (int)s0 + grp * kStageKeys, kw0 = k0 + 16 * wq, kend = (int)s1 - 1;
+            r_stage = first_kept_pair(sw, H, Lq - (k0 + kStageKeys - 1 < kend ? k0 + kStageKeys - 1 : kend));
+            r_warp = first_kept_pair(sw, H, Lq - (kw0 + 15 < kend ? kw0 + 15 : kend));
+            r_keep = first_kept_pair(sw, H, Lq - kw0);
+        }
         for (int it = grp; it < nstage && ok; it += kGroups) {
             const int st = it % kStages;
             const int k0 = (int)s0 + it * kStageKeys;

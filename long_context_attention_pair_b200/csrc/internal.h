@@ -19,6 +19,34 @@ bool theta_valid(int D, const double *theta);
 int window_table_theta(int D, const double *theta, double k, int64_t N, int64_t *w);
 int pruned_terms_theta(int64_t N, int D, const double *theta, double k, atflash_terms *out);
 
+// Programmatic dependent launch (sm_90 and later).  A kernel launched with
+// launch_dependent() may be scheduled while the previous kernel in the stream
+// still runs; it must call pdl_wait() before it touches anything that kernel
+// writes (the wait returns once the previous kernel has completed and its
+// memory operations are visible; in a kernel launched without the attribute it
+// returns at once).  pdl_allow_dependents() lets the dependent launch begin
+// before the calling kernel ends.
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+template <typename... KArgs, typename... Args>
+static inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                           cudaStream_t s, Args... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+#endif
+
 // Per-call constants shared by every kernel of one call.
 struct WindowParams {
     int H;                      // D/2 pairs

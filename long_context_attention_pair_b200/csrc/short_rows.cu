@@ -154,6 +154,9 @@ __global__ void __launch_bounds__(kThreads) short_rows_kernel(const __grid_const
     int64_t seq_len = 0, tokbase = 0, n0 = 0;
     int bz = b;
     if constexpr (kDecode) {
+        // A programmatic dependent of the merge, whose output rows it overwrites;
+        // every CTA waits, so that this kernel never completes before the merge.
+        pdl_wait();
         seq_len = a.seqlens[b];
         if (seq_len < 1 || seq_len > kTile || seq_len > a.N) return;
     } else {
@@ -341,8 +344,13 @@ static cudaError_t launch(const Args &a, const WindowParams &wp, dim3 grid, cuda
     cudaError_t e = cudaFuncSetAttribute(short_rows_kernel<D, kDecode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem);
     if (e != cudaSuccess) return e;
-    short_rows_kernel<D, kDecode><<<grid, kThreads, smem, s>>>(a, wp);
-    return cudaGetLastError();
+    if constexpr (kDecode) {
+        // After the merge, as its programmatic dependent.
+        return launch_dependent(short_rows_kernel<D, kDecode>, grid, dim3(kThreads), smem, s, a, wp);
+    } else {
+        short_rows_kernel<D, kDecode><<<grid, kThreads, smem, s>>>(a, wp);
+        return cudaGetLastError();
+    }
 }
 
 }  // namespace sr

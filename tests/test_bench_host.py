@@ -61,12 +61,16 @@ def test_captured_traffic_is_reported_only_for_its_own_workload():
     assert bench.decode_traffic("decode_128k", 1 << 17) is None
     # natural layouts read the whole cache: the capture scales with L; packed does not
     rec = bench.DECODE_TRAFFIC["decode_1m"]
-    same = rec["source_sha1"] == bench.kernel_sha1("decode_tc.cu")
+    same = rec["source_sha1"] == bench.kernel_sha1(*bench.DECODE_SOURCES)
     got = bench.decode_traffic("decode_1m", 1 << 20)
     assert (got == round(rec["bytes_per_launch"] * (1 << 20) / rec["captured_L"])) if same else got is None
     assert bench.decode_traffic("decode_1m_packed", 1 << 20) is None
     pk = bench.DECODE_TRAFFIC["decode_1m_packed"]
     assert (bench.decode_traffic("decode_1m_packed", pk["captured_L"]) == pk["bytes_per_launch"]) == same
+    # a sweep over the number of sequences: the natural layout scales with B * L, packed is not reported
+    got1 = bench.decode_traffic("decode_1m", 1 << 19, B=1)
+    assert (got1 == round(rec["bytes_per_launch"] * (1 << 19) / (4 * rec["captured_L"]))) if same else got1 is None
+    assert bench.decode_traffic("decode_1m_packed", pk["captured_L"], B=1) is None
 
 
 def test_tile_flops_sum_to_the_dense_retained_flops():

@@ -94,7 +94,7 @@ def test_noalloc_decode_matches_workspace_decode_twice(in_name, layout, out_name
 
 def test_noalloc_rejects_problems_beyond_the_fixed_scratch():
     B, Hq, Hkv, D = 16, 64, 4, 128
-    Nmax = 1 << 20  # 16*64*512*(128+2)*4 bytes of split states: far above the limit
+    Nmax = 1 << 20  # 16*64*256*(128+2)*4 bytes of split states: far above the limit
     assert atf.decode_workspace_bytes(B, Hq, Hkv, Nmax, D) > LIMIT
     fake = torch.empty(64, dtype=torch.uint8, device="cuda")  # never touched: rejected first
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
