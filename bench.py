@@ -299,11 +299,11 @@ TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98543616,
 # a sector), so their traffic grows in proportion to B * L and is scaled to the
 # line's; the packed layout's kept share depends on L, so it is reported only at
 # the captured length and the workload's own B.
-DECODE_TRAFFIC = {"decode_1m": {"captured_L": 131072, "bytes_per_launch": 1078800128, "proportional_to_L": True,
-                                "source_sha1": "3f0aa78370ba9c79bdc31255877b0817885b25c3"},
-                  "decode_1m_packed": {"captured_L": 131072, "bytes_per_launch": 897253632,
+DECODE_TRAFFIC = {"decode_1m": {"captured_L": 131072, "bytes_per_launch": 1078782976, "proportional_to_L": True,
+                                "source_sha1": "f90fa0ad91c3ec30c6ce5b524acae257bf566d1f"},
+                  "decode_1m_packed": {"captured_L": 131072, "bytes_per_launch": 897764352,
                                        "proportional_to_L": False,
-                                       "source_sha1": "3f0aa78370ba9c79bdc31255877b0817885b25c3"}}
+                                       "source_sha1": "f90fa0ad91c3ec30c6ce5b524acae257bf566d1f"}}
 
 
 def parse():
