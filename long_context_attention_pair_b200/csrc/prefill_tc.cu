@@ -20,19 +20,23 @@
 // CTA = one 128-row query tile of TWO query heads of the same GQA group: both
 // heads read the same K/V tiles at the same distances, so they share every
 // load, every pruned-chunk decision and every boundary pair, while their two
-// softmax warpgroups ping-pong with the tensor core.  12 warps:
-//   warps 0-3 / 4-7  softmax of head 0 / head 1: one TMEM lane quarter each;
-//                    boundary fix-up, causal mask, online softmax in the log2
-//                    domain, P (bf16) into TMEM, O rescale (only when the
-//                    running max grows by more than 2^8), epilogue O / l
-//   warp 8           TMA producer (Q~ once; K~ chunks and V per key tile)
-//   warp 9           TMEM owner and QK issuer: S_h = Q~_h K~^T (smem x smem)
-//   warp 10          zeroes the fully-pruned pairs of the first loaded K~ chunk
+// softmax warps ping-pong with the tensor core.  20 warps:
+//   warps 0-7 / 8-15 softmax of head 0 / head 1: warp 4 hc + q4 of a head takes
+//                    TMEM lane quarter q4 (32 query rows) and S columns
+//                    [64 hc, 64 hc + 64) of the key tile; the two warps of a row
+//                    exchange their partial row maxima once per tile (and their
+//                    partial sums at the end).  Boundary fix-up, causal mask,
+//                    online softmax in the log2 domain, P (bf16) into TMEM, O
+//                    rescale (only when the running max grows by more than 2^8)
+//                    and the epilogue, each on the warp's half of the columns
+//   warp 16          TMA producer (Q~ once; K~ chunks and V per key tile)
+//   warp 17          TMEM owner and QK issuer: S_h = Q~_h K~^T (smem x smem)
+//   warp 18          zeroes the fully-pruned pairs of the first loaded K~ chunk
 //                    and stages the tile's boundary pairs as fp32 for the fix-up
-//   warp 11          PV issuer: O_h += P_h V (P from TMEM, V from smem)
+//   warp 19          PV issuer: O_h += P_h V (P from TMEM, V from smem)
 // For D = 64 with no pair pruned anywhere the launcher takes the one-head form
-// instead: 8 warps (softmax 0-3, then producer, QK, fix-up, PV), 256 TMEM
-// columns and two K/V stages, so that two CTAs share an SM.
+// instead: 8 warps (softmax 0-3 over whole rows, then producer, QK, fix-up,
+// PV), 256 TMEM columns and two K/V stages, so that two CTAs share an SM.
 // TMEM columns: as in Cfg below.
 // Every mbarrier wait is bounded in time; on expiry the CTA records
 // ATFLASH_ERR_TIMEOUT in the device status word, lets its copies land, drains
@@ -51,12 +55,24 @@ constexpr int kBM = 128;
 constexpr int kBN = 128;
 // NH query heads per CTA (2: one CTA per SM, the heads share every K/V tile; 1:
 // two CTAs per SM, which run out of phase so one CTA's exp2 pass overlaps the
-// other's loads, waits and stores).  Warps: 4*NH softmax, then producer, QK
-// issuer, fix-up and PV issuer.
-template <int NH>
+// other's loads, waits and stores).  CH softmax warps share each row's 128
+// columns (2: with window pruning, where the boundary subtraction and the
+// shorter per-warp passes pay for a per-tile exchange of partial row maxima;
+// 1: whole rows, which measured faster without pruning).  Warps: 4*NH*CH
+// softmax, then producer, QK issuer, fix-up and PV issuer.  Registers: every
+// thread gets LaunchRegs at launch; the four other warps drop to OtherRegs and
+// the softmax warps rise to SoftRegs, which must fit the launch's total
+// (checked here and, against the compiled kernel, at launch).
+template <int NH, int CH>
 struct Warps {
-    static constexpr int Threads = 32 * (4 * NH + 4);
-    static constexpr int Producer = 4 * NH, Mma = 4 * NH + 1, Fix = 4 * NH + 2, Pv = 4 * NH + 3;
+    static constexpr int Soft = 4 * NH * CH;
+    static constexpr int Threads = 32 * (Soft + 4);
+    static constexpr int Producer = Soft, Mma = Soft + 1, Fix = Soft + 2, Pv = Soft + 3;
+    static constexpr int LaunchRegs = 65536 / (Threads * (3 - NH)) / 8 * 8;
+    static constexpr int OtherRegs = (NH == 2 && CH == 1) ? 96 : 56;
+    static constexpr int SoftRegs = CH == 2 ? 104 : 200;
+    static_assert(NH == 2 || CH == 1, "the one-head form keeps whole rows");
+    static_assert(32 * Soft * SoftRegs + 128 * OtherRegs <= Threads * LaunchRegs, "register split exceeds the launch");
 };
 constexpr uint32_t kChunkBytes = kBN * 32;  // 128 rows x 16 bf16 (one K-step)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
@@ -79,7 +95,8 @@ struct Cfg {
     static constexpr int OffBnd = OffV + VS * VBytes;                 // [KS][kMaxStagedPairs][64] float4
     static constexpr int BndBytes = kMaxStagedPairs * 64 * 16;
     static constexpr int OffCtl = OffBnd + KS * BndBytes;
-    static constexpr int Total = OffCtl + 2048;
+    static constexpr int CtlBytes = 6144;
+    static constexpr int Total = OffCtl + CtlBytes;
     static constexpr int Request = Total + 1024;
     // TMEM, two heads: D = 64: S0 [0,128), S1 [128,256), O0, O1 [256,384), P0, P1 [384,512).
     //                  D = 128: one S [0,128) shared by the two heads in turn, P0 [128,192),
@@ -102,9 +119,11 @@ struct Ctl {
     uint64_t v_full[VS], v_empty[VS];
     uint64_t s_full[2], s_read[2], p_full[2], o_done[2];
     uint64_t drain;
+    uint64_t xbar[2][4];             // (head, lane quarter): both column halves have posted
     uint32_t tmem_base;
     int abort_flag;
     int w[kMaxPairs];
+    float xval[2][4][2][2][32];      // (head, quarter, tile parity, column half, lane)
 };
 
 // Byte offset of 32-bit word `word` (0..7) of row `row` in a 128 x 32 B chunk
@@ -189,14 +208,14 @@ __device__ __forceinline__ bool wait_drain(uint64_t *bar, uint32_t parity, uint6
 // and N is the longest sequence.  Otherwise q/k/v/out are [B][N][H][D].
 // kMasked: token-level block selection, block_mask [B][Hkv][T][T] (T query /
 // key tiles of 128), entry (b, g, i, j) != 0 keeps key tile j for query tile i.
-template <int D, bool kVarlen, int NH, bool kMasked>
-__global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
+template <int D, bool kVarlen, int NH, bool kMasked, int CH>
+__global__ void __launch_bounds__(Warps<NH, CH>::Threads, 3 - NH)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ WindowParams wp,
                       void *out, int out_f32, float *lse, int64_t N, int Hq, int Hkv, int *status,
                       uint64_t limit_ns, const int32_t *cu_seqlens, int64_t total, const uint8_t *block_mask) {
     using F = Cfg<D, NH>;
-    using W = Warps<NH>;
+    using W = Warps<NH, CH>;
     constexpr int kThreads = W::Threads;
     constexpr int kWarpProducer = W::Producer, kWarpMma = W::Mma, kWarpFix = W::Fix, kWarpPv = W::Pv;
     constexpr uint32_t kTmemCols = F::TmemCols;
@@ -210,6 +229,7 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
     uint8_t *sV = smem + F::OffV;
     float4 *sBnd = reinterpret_cast<float4 *>(smem + F::OffBnd);
     Ctl<KS, VS> *ctl = reinterpret_cast<Ctl<KS, VS> *>(smem + F::OffCtl);
+    static_assert(sizeof(Ctl<KS, VS>) <= F::CtlBytes, "control block outgrew its space");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_qt = (int)((N + kBM - 1) / kBM);
@@ -247,7 +267,7 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
         for (int s = 0; s < KS; ++s) {
             mbar_init(&ctl->k_full[s], 1);
             mbar_init(&ctl->k_ready[s], 1);
-            mbar_init(&ctl->k_empty[s], 1 + 4 * nwg);
+            mbar_init(&ctl->k_empty[s], 1 + 4 * CH * nwg);
         }
         for (int s = 0; s < VS; ++s) {
             mbar_init(&ctl->v_full[s], 1);
@@ -255,11 +275,13 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&ctl->s_full[s], 1);
-            mbar_init(&ctl->s_read[s], 4);
-            mbar_init(&ctl->p_full[s], 4);
+            mbar_init(&ctl->s_read[s], 4 * CH);
+            mbar_init(&ctl->p_full[s], 4 * CH);
             mbar_init(&ctl->o_done[s], 1);
         }
         mbar_init(&ctl->drain, 2);  // one commit from each issuing warp
+        for (int t = 0; t < 2; ++t)
+            for (int q = 0; q < 4; ++q) mbar_init(&ctl->xbar[t][q], CH);
         ctl->abort_flag = 0;
         fence_mbar_init();
     }
@@ -275,17 +297,12 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
     const int *w = ctl->w;
     WaitCtl wc{&ctl->abort_flag, status, limit_ns, 0};
 
-    // Register split.  Two heads: the launch gives every thread 168 registers
-    // (384 x 168 = 64512); warpgroup 2 (producer, MMA, fix-up, PV) drops to 96 and
-    // the two softmax warpgroups rise to 200: 128 x 96 + 256 x 200 = 63488 <= 64512.
-    // One head (two CTAs per SM): 128 registers at launch (256 x 128 = 32768);
-    // warpgroup 1 drops to 56 and the softmax warpgroup rises to 200:
-    // 128 x 56 + 128 x 200 = 32768.
-    if constexpr (NH == 2) {
-        if (warp >= 8) setmaxnreg_dec<96>();
-    } else {
-        if (warp >= 4) setmaxnreg_dec<56>();
-    }
+    // Register split (Warps): two heads, split rows: 640 threads at 96 registers
+    // (61440); the last warpgroup (producer, MMA, fix-up, PV) drops to 56 and the
+    // four softmax warpgroups rise to 104: 128 x 56 + 512 x 104 = 60416.  Two
+    // heads, whole rows: 384 threads at 168 (64512); 128 x 96 + 256 x 200 = 63488.
+    // One head (two CTAs per SM): 256 threads at 128 (32768); 128 x 56 + 128 x 200.
+    if (warp >= W::Soft) setmaxnreg_dec<W::OtherRegs>();
     if (warp == kWarpProducer) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -446,21 +463,28 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
             if (ok && lane == 0) umma_commit(&ctl->v_empty[vs]);
             __syncwarp();
         }
-    } else if (warp < 4 * NH) {
+    } else if (warp < W::Soft) {
         // ------------------------------------------------------------- softmax
-        setmaxnreg_inc<200>();
-        const int t = warp >> 2;  // which head of the pair
+        setmaxnreg_inc<W::SoftRegs>();
+        constexpr int kCols = kBN / CH;    // S columns per warp
+        constexpr int kOCols = D / CH;     // O columns per warp (rescale, epilogue)
+        const int t = warp / (4 * CH);     // which head of the pair
         if (t < nwg) {
-            const int q4 = warp & 3;
+            const int q4 = warp & 3, hc = (warp >> 2) % CH;
+            const int c0 = hc * kCols;     // this warp's first column of the key tile
             const int row = q4 * 32 + lane;
             const int64_t n = n0 + row;
             const int hq = h0 + t;
             const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-            const uint32_t tS = tmem + (t ? F::TmemS1 : F::TmemS0) + lane_off;
-            const uint32_t tP = tmem + (t ? F::TmemP1 : F::TmemP0) + lane_off;
-            const uint32_t tO = tmem + (t ? F::TmemO1 : F::TmemO0) + lane_off;
+            const uint32_t tS = tmem + (t ? F::TmemS1 : F::TmemS0) + lane_off + c0;
+            const uint32_t tP = tmem + (t ? F::TmemP1 : F::TmemP0) + lane_off + c0 / 2;
+            const uint32_t tO = tmem + (t ? F::TmemO1 : F::TmemO0) + lane_off + hc * kOCols;
             const uint8_t *sQt = sQ + t * F::QBytes;
             const float scale_log2 = 1.4426950408889634f * rsqrtf((float)D);
+            // The two warps of a row post partial values here (parity of the tile
+            // count: a slot is rewritten only after the partner has passed the
+            // next exchange, hence has read it).
+            uint64_t *xbar = &ctl->xbar[t][q4];
             float m_used = -INFINITY, lrun = 0.f;
             wc.site = 8;
             bool ok = mbar_wait_warp(&ctl->q_full, 0, wc);  // Q~ rows are read for the boundary fix-up
@@ -471,15 +495,21 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                 const int ks = it % KS;
                 const int64_t m0 = (int64_t)j * kBN;
                 const Band bd = bw.at(w, n0, m0);
-                float s[kBN];
+                float s[kCols];
                 wc.site = 9;
                 if (!(ok = mbar_wait_warp(&ctl->s_full[t], it & 1, wc))) break;
                 tc_fence_after();
                 if ((bd.r_lo >> 3) < C) {
-                    // The whole row in one 128-column load in the two-head kernel, two 64-column
-                    // loads in the one-head kernel (128 registers at launch); both measured faster
-                    // than four loads of 32 columns.
-                    if constexpr (NH == 2) {
+                    // One load of the warp's columns; two of 64 for a whole row in the
+                    // one-head kernel (launched with 128 registers).  Both measured faster
+                    // than loads of 32 columns.
+                    if constexpr (kCols == 64) {
+                        uint32_t ra[64];
+                        tmem_ld_32x32b_x64(tS, ra);
+                        tmem_ld_wait(ra);
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(ra[i]);
+                    } else if constexpr (NH == 2) {
                         uint32_t ra[128];
                         tmem_ld_32x32b_x128(tS, ra);
                         tmem_ld_wait(ra);
@@ -499,7 +529,7 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                     }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < kBN; ++i) s[i] = 0.f;
+                    for (int i = 0; i < kCols; ++i) s[i] = 0.f;
                 }
                 // S is in registers: the MMA may reuse its columns.
                 tc_fence_before();
@@ -516,9 +546,9 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                     if (!(ok = mbar_wait_warp(&ctl->k_ready[ks], (it / KS) & 1, wc))) break;
                     const float4 *bst = sBnd + ks * (kMaxStagedPairs * 64);
                     for (int r = bd.r_lo; r < bd.r_full; ++r) {
-                        const int lim = (int)(n - m0 - (int64_t)w[r]);
+                        const int lim = (int)(n - m0 - (int64_t)w[r]);  // cells jj < lim drop pair r
                         const int lim_max = __reduce_max_sync(0xffffffffu, lim);
-                        if (lim_max <= 0) continue;
+                        if (lim_max <= c0) continue;  // none of this warp's columns
                         const uint32_t qw =
                             *reinterpret_cast<const uint32_t *>(sQt + (r >> 3) * kChunkBytes + sw32_off(row, r & 7));
                         const float2 qa2 = make_float2(bf16lo(qw), bf16lo(qw));
@@ -529,16 +559,16 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                             // blocks every row of the warp prunes in full measured slower (the
                             // larger correction code cost more than the saved compares).
 #pragma unroll
-                            for (int cc = 0; cc < 4; ++cc) {
-                                if (32 * cc < lim_max) {
+                            for (int cc = 0; cc < kCols / 32; ++cc) {
+                                if (c0 + 32 * cc < lim_max) {
 #pragma unroll
                                     for (int i = 0; i < 16; ++i) {
-                                        const int jj = 32 * cc + 2 * i;
-                                        const float4 kv = kb[16 * cc + i];
+                                        const int jl = 32 * cc + 2 * i, jj = c0 + jl;
+                                        const float4 kv = kb[jj / 2];
                                         const float2 t = fma2(qa2, make_float2(kv.x, kv.y),
                                                               mul2(qb2, make_float2(kv.z, kv.w)));
-                                        if (jj < lim) s[jj] -= t.x;
-                                        if (jj + 1 < lim) s[jj + 1] -= t.y;
+                                        if (jj < lim) s[jl] -= t.x;
+                                        if (jj + 1 < lim) s[jl + 1] -= t.y;
                                     }
                                 }
                             }
@@ -547,15 +577,15 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                             const float qa = qa2.x, qb = qb2.x;
                             const uint8_t *kch = sK + ks * F::KBytes + (r >> 3) * kChunkBytes;
 #pragma unroll
-                            for (int cc = 0; cc < 4; ++cc) {
-                                if (32 * cc < lim_max) {
+                            for (int cc = 0; cc < kCols / 32; ++cc) {
+                                if (c0 + 32 * cc < lim_max) {
 #pragma unroll
                                     for (int i = 0; i < 32; ++i) {
-                                        const int jj = 32 * cc + i;
+                                        const int jl = 32 * cc + i, jj = c0 + jl;
                                         if (jj < lim) {
                                             const uint32_t kw =
                                                 *reinterpret_cast<const uint32_t *>(kch + sw32_off(jj, r & 7));
-                                            s[jj] -= qa * bf16lo(kw) + qb * bf16hi(kw);
+                                            s[jl] -= qa * bf16lo(kw) + qb * bf16hi(kw);
                                         }
                                     }
                                 }
@@ -569,18 +599,30 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                 // of 3-input max); the 1/sqrt(D) * log2(e) scale is folded into the exp.
                 if (j == qt) {
 #pragma unroll
-                    for (int jj = 0; jj < kBN; ++jj)
-                        if (jj > row) s[jj] = -INFINITY;
+                    for (int jl = 0; jl < kCols; ++jl)
+                        if (c0 + jl > row) s[jl] = -INFINITY;
                 }
                 float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-                for (int jj = 0; jj < kBN; jj += 8) {
+                for (int jj = 0; jj < kCols; jj += 8) {
                     mx0 = max3(mx0, s[jj], s[jj + 1]);
                     mx1 = max3(mx1, s[jj + 2], s[jj + 3]);
                     mx2 = max3(mx2, s[jj + 4], s[jj + 5]);
                     mx3 = max3(mx3, s[jj + 6], s[jj + 7]);
                 }
-                const float tile_max = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * scale_log2;
+                float raw_max = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+                if constexpr (CH == 2) {
+                    // The row's maximum over both column halves, so that both warps take
+                    // the same running max (P of one row must share it).
+                    float *slot = ctl->xval[t][q4][it & 1][0];
+                    slot[hc * 32 + lane] = raw_max;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(xbar);
+                    wc.site = 13;
+                    if (!(ok = mbar_wait_warp(xbar, it & 1, wc))) break;
+                    raw_max = fmaxf(raw_max, slot[(hc ^ 1) * 32 + lane]);
+                }
+                const float tile_max = raw_max * scale_log2;
                 // Keep the previous (stale) max unless the row max grew by more than
                 // 2^8: the final O / l uses the same max, so the result is exact.
                 const bool need = tile_max > m_used + kRescaleThreshold;
@@ -591,9 +633,9 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                 const float2 mneg = make_float2(-m_used, -m_used);
                 const float2 sc2 = make_float2(scale_log2, scale_log2);
                 float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
-                uint32_t pk[64];
+                uint32_t pk[kCols / 2];
 #pragma unroll
-                for (int i = 0; i < 64; i += 2) {
+                for (int i = 0; i < kCols / 2; i += 2) {
                     float2 xa = fma2(make_float2(s[2 * i], s[2 * i + 1]), sc2, mneg);
                     float2 xb = fma2(make_float2(s[2 * i + 2], s[2 * i + 3]), sc2, mneg);
                     xa.x = fast_exp2(xa.x);
@@ -615,7 +657,7 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                 }
                 if (rescale) {
 #pragma unroll 1
-                    for (int cc = 0; cc < D / 32; ++cc) {
+                    for (int cc = 0; cc < kOCols / 32; ++cc) {
                         uint32_t r[32];
                         tmem_ld_32x32b_x32(tO + cc * 32, r);
                         tmem_ld_wait(r);
@@ -624,13 +666,10 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                         tmem_st_32x32b_x32(tO + cc * 32, r);
                     }
                 }
-                // P_t (bf16 pairs) into its own 64 columns.
-                {
-                    uint32_t (&pa)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-                    uint32_t (&pb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-                    tmem_st_32x32b_x32(tP + 0, pa);
-                    tmem_st_32x32b_x32(tP + 32, pb);
-                }
+                // This warp's part of P_t (bf16 pairs of its columns).
+#pragma unroll
+                for (int cc = 0; cc < kCols / 64; ++cc)
+                    tmem_st_32x32b_x32(tP + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * cc]));
                 tmem_st_wait();
                 const float2 ls = add2(l0, l1);
                 lrun = lrun * alpha + (ls.x + ls.y);
@@ -642,12 +681,24 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                 wc.site = 12;
                 ok = mbar_wait_warp(&ctl->o_done[t], (it - 1) & 1, wc);
             }
+            if constexpr (CH == 2) {
+                // The row's sum over both column halves (one more exchange).
+                if (ok) {
+                    float *slot = ctl->xval[t][q4][it & 1][0];
+                    slot[hc * 32 + lane] = lrun;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(xbar);
+                    wc.site = 13;
+                    ok = mbar_wait_warp(xbar, it & 1, wc);
+                    if (ok) lrun += slot[(hc ^ 1) * 32 + lane];
+                }
+            }
             if (ok) {
                 tc_fence_after();
                 const float inv = 1.f / lrun;
-                const size_t o = ((size_t)((int64_t)bz * nrows + tokbase + n) * Hq + hq) * D;
+                const size_t o = ((size_t)((int64_t)bz * nrows + tokbase + n) * Hq + hq) * D + hc * kOCols;
 #pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
+                for (int cc = 0; cc < kOCols / 32; ++cc) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(tO + cc * 32, r);
                     tmem_ld_wait(r);
@@ -677,7 +728,7 @@ __global__ void __launch_bounds__(Warps<NH>::Threads, 3 - NH)
                         }
                     }
                 }
-                if (lse && n < seq_len)
+                if (lse && hc == 0 && n < seq_len)
                     lse[((size_t)bz * Hq + hq) * nrows + tokbase + n] = (m_used + __log2f(lrun)) * 0.69314718055994531f;
             }
         }
@@ -746,41 +797,51 @@ cudaError_t launch_prefill_tc(const void *qpack, const void *kpack, const void *
     const int num_qt = (int)((p.N + tc::kBM - 1) / tc::kBM);
     const int G = p.Hq / p.Hkv;
     cudaError_t e;
-#define ATF_PREFILL_TC_M(DD, VL, NHH, MK)                                                                        \
+#define ATF_PREFILL_TC_M(DD, VL, NHH, MK, CHH)                                                                   \
     do {                                                                                                         \
         const int smem = tc::Cfg<DD, NHH>::Request;                                                             \
         dim3 grid((unsigned)num_qt, (unsigned)(p.B * p.Hkv * ((G + NHH - 1) / NHH)));                          \
-        e = cudaFuncSetAttribute(tc::prefill_tc_kernel<DD, VL, NHH, MK>,                                        \
+        e = cudaFuncSetAttribute(tc::prefill_tc_kernel<DD, VL, NHH, MK, CHH>,                                        \
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                             \
         if (e != cudaSuccess) return e;                                                                          \
-        tc::prefill_tc_kernel<DD, VL, NHH, MK><<<grid, tc::Warps<NHH>::Threads, smem, s>>>(                     \
+        /* The in-kernel register split assumes this launch count: refuse to run otherwise. */                  \
+        cudaFuncAttributes fa;                                                                                   \
+        if ((e = cudaFuncGetAttributes(&fa, tc::prefill_tc_kernel<DD, VL, NHH, MK, CHH>)) != cudaSuccess) return e;  \
+        if (fa.numRegs != tc::Warps<NHH, CHH>::LaunchRegs) return cudaErrorInvalidConfiguration;                      \
+        tc::prefill_tc_kernel<DD, VL, NHH, MK, CHH><<<grid, tc::Warps<NHH, CHH>::Threads, smem, s>>>(                     \
             tq, tk, tv, wp, out, out_f32, lse, p.N, p.Hq, p.Hkv, status, wait_limit_ns, cu_seqlens, total,       \
             block_mask);                                                                                         \
     } while (0)
     // Block-selected launches (never varlen) take their own instantiations, so that
     // the dense kernels' code is what it was.
-#define ATF_PREFILL_TC(DD, VL, NHH)                                                                              \
+#define ATF_PREFILL_TC(DD, VL, NHH, CHH)                                                                         \
     do {                                                                                                         \
         if constexpr (!VL) {                                                                                     \
             if (masked) {                                                                                        \
-                ATF_PREFILL_TC_M(DD, false, NHH, true);                                                          \
+                ATF_PREFILL_TC_M(DD, false, NHH, true, CHH);                                                     \
                 break;                                                                                           \
             }                                                                                                    \
         }                                                                                                        \
-        ATF_PREFILL_TC_M(DD, VL, NHH, false);                                                                    \
+        ATF_PREFILL_TC_M(DD, VL, NHH, false, CHH);                                                               \
     } while (0)
+    // No pair pruned anywhere (k = inf, or windows covering the longest sequence).
+    const bool unpruned = (int64_t)wp.w[0] >= p.N - 1;
     if (p.D == 128) {
-        if (varlen) ATF_PREFILL_TC(128, true, 2); else ATF_PREFILL_TC(128, false, 2);
-    } else if (p.D == 64) {
-        // No pair pruned anywhere (k = inf, or windows covering the longest sequence):
-        // one head per CTA, two CTAs per SM measured faster (no boundary work to share
-        // between heads).  With pruning, two heads per CTA share every K~ tile's
-        // zeroing and boundary staging and measured faster.
-        const bool unpruned = (int64_t)wp.w[0] >= p.N - 1;
+        // Two heads per CTA; each row split between two softmax warps only with pruning
+        // (without it the whole-row form measured faster).
         if (unpruned) {
-            if (varlen) ATF_PREFILL_TC(64, true, 1); else ATF_PREFILL_TC(64, false, 1);
+            if (varlen) ATF_PREFILL_TC(128, true, 2, 1); else ATF_PREFILL_TC(128, false, 2, 1);
         } else {
-            if (varlen) ATF_PREFILL_TC(64, true, 2); else ATF_PREFILL_TC(64, false, 2);
+            if (varlen) ATF_PREFILL_TC(128, true, 2, 2); else ATF_PREFILL_TC(128, false, 2, 2);
+        }
+    } else if (p.D == 64) {
+        // Unpruned: one head per CTA, two CTAs per SM measured faster (no boundary work
+        // to share between heads).  With pruning, two heads per CTA share every K~
+        // tile's zeroing and boundary staging, with split rows.
+        if (unpruned) {
+            if (varlen) ATF_PREFILL_TC(64, true, 1, 1); else ATF_PREFILL_TC(64, false, 1, 1);
+        } else {
+            if (varlen) ATF_PREFILL_TC(64, true, 2, 2); else ATF_PREFILL_TC(64, false, 2, 2);
         }
     } else {
         return cudaErrorInvalidValue;
