@@ -289,8 +289,8 @@ KERNELS_PER_STEP = 7
 # DRAM bytes per launch of the tcgen05 prefill kernel, from one ncu capture per
 # workload.  Valid only while the kernel source hashes to `source_sha1`;
 # otherwise the line reports null.
-TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 98543616,
-           "source_sha1": "0d19d32cb15f5f9de5107841ea5bf3503b043c96"}
+TRAFFIC = {"workload": "qwen05b_32k", "bytes_per_launch": 99928064,
+           "source_sha1": "9c36dbd1d5526ea2ee85f8ca868407a38a2cf948"}
 # DRAM bytes per launch of the decode kernel (split states included, merge not),
 # from an ncu capture of the same workload at a shorter cache length
 # `captured_L`; valid while decode_tc.cu and decode.cu (the split heuristic)
