@@ -72,6 +72,43 @@ def test_bf16_prefill_matches_oracle(oracle, B, N, D, Hq, Hkv, base, kwin):
     P.check(P.host(lse), rlse.transpose(0, 2, 1), "bf16", "bf16 lse")
 
 
+# One key whose score exceeds every other score of its rows by >= 15 (natural
+# units) sits in a chosen column of its key tile: rows after it see their running
+# max jump by > 2^8 at that tile (the O rescale), first in the softmax warp that
+# holds that column (with pruning two warps share a row and must adopt the same
+# max).  The query and that key share a direction in the pairs that turn less
+# than 0.5 rad over the sequence (never pruned at these k); every other key is
+# zero there.  The dominant key takes nearly all the weight, so the output does
+# not depend on the bf16 rounding of the large score.
+@pytest.mark.parametrize("D,base,kwin,m_star", [
+    (64, 1e6, 8.0, 128 * 3 + 100),   # column 100: the second half of the tile's row
+    (64, 1e6, 8.0, 128 * 3 + 20),    # column 20: the first half
+    (128, 5e5, 16.0, 128 * 5 + 90),
+    (128, 5e5, 16.0, 128 * 7 + 40),  # the diagonal tile of the last query tile
+])
+def test_bf16_row_max_jump_in_one_column_half(oracle, D, base, kwin, m_star):
+    N, Hq, Hkv = 1024, 2, 1
+    q, k, v = inputs(8, 1, N, Hq, Hkv, D, "bf16")
+    low = [r for r in range(D // 2) if base ** (-2 * r / D) * N < 0.5]
+    assert len(low) >= 14 and min(atf.window_table(D, base, kwin, N)[r] for r in low) == N - 1
+    q[..., low] = 2.0
+    k[..., low] = 0.0
+    k[0, m_star, :, low] = 6.0
+    out, lse = atf.prefill(q, k, v, base, kwin, out_dtype=torch.float32, return_lse=True)
+    torch.cuda.synchronize()
+    ref, rlse = oracle.prefill(P.host(q), P.host(k), P.host(v), base, kwin, want_lse=True)
+    # the dominant key carries almost all the weight of every later row
+    vh = P.host(v)[0, m_star, 0]
+    assert np.abs(ref[0, m_star + 1:, 0] - vh).max() < 0.01
+    P.check(P.host(out), ref, "bf16", f"row max jump D={D} m*={m_star}")
+    # The log-sum-exp of a later row is about the dominant score itself (15-26 here).
+    # Its terms are all positive, so rounding the rotated q~ and k~ to bf16 (relative
+    # 2^-9 each) moves it by up to 2^-8 of its size: the bar is relative there.
+    got_lse, ref_lse = P.host(lse), rlse.transpose(0, 2, 1)
+    assert np.all(np.abs(got_lse - ref_lse) <= 1e-2 + 2.0 ** -8 * np.abs(ref_lse))
+    assert atf.device_status() == 0
+
+
 def test_bf16_output_rounding(oracle):
     # bf16 output: oracle value rounded to bf16, within 1e-2 plus half a bf16 ulp.
     q, k, v = inputs(3, 1, 600, 2, 1, 128, "bf16")
