@@ -261,7 +261,10 @@ int atflash_decode_paged(const void *q, const void *kpages, const void *vpages, 
                          int page_size, int D, double rope_base, double k_window, int kcache_rotated, int kv_layout,
                          int out_dtype, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
-/* Device scratch bytes atflash_decode needs (0 on invalid arguments). */
+/* Device scratch bytes atflash_decode needs (0 on invalid arguments): one split
+ * state of D + 2 floats per (sequence, query head, split).  A split is 256 to
+ * 4096 keys, a multiple of 64, chosen so that the B * Hkv * splits CTAs come
+ * close to, without passing, a whole number of waves of 148 SMs x 3 CTAs. */
 size_t atflash_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int D);
 
 /*
@@ -269,7 +272,10 @@ size_t atflash_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t Nmax, int 
  * (README "Numbers"/"Using the ports": the window is one more condition on
  * which K elements are loaded).  Split-KV: each CTA streams one slice of one
  * sequence's cache, loading only the K dims kept at that slice's distances,
- * and a second kernel merges the slices' softmax states.
+ * and a second kernel merges the slices' softmax states.  The merge (and, for
+ * bf16 caches, the fp32 short-row step) is launched on `stream` as a
+ * programmatic dependent of the kernel before it; the call captures into a
+ * CUDA graph as one chain.
  *   q              [B][Hq][D]        un-rotated query of each sequence
  *   kcache, vcache keys (un-rotated unless kcache_rotated) and values, in
  *                  kv_layout ATFLASH_KV_HND [B][Hkv][Nmax][D] or

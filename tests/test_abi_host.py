@@ -343,3 +343,21 @@ def test_short_rows_step_argument_errors(L):
     assert f(U, A, A, A, 1, 2, 1, 256, 64, 1e4, 1.0, atf.BF16, None, None) == -6      # alignment
     g = L.atflash_prefill_short_rows_theta
     assert g(A, A, A, A, 1, 2, 1, 256, 64, None, 1.0, atf.BF16, None, None) == -1     # no table
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N", [
+    (1, 28, 4, 8192), (1, 28, 4, 1 << 19), (4, 28, 4, 1 << 20), (16, 28, 4, 1 << 17), (1, 14, 2, 32768),
+    (1, 24, 8, 131072), (3, 8, 1, 1 << 20), (1, 1, 1, 256), (1, 4, 1, 1000), (64, 32, 8, 4096)])
+def test_decode_splits_fill_whole_waves(B, Hq, Hkv, N):
+    # The split count behind the workspace size: splits of 256..4096 keys (so at
+    # least ceil(N/4096) and at most ceil(N/256) of them), and the B*Hkv*splits
+    # CTAs never pass the whole number of 148 x 3 waves that 4096-key splits need.
+    D = 128
+    ws = atf.decode_workspace_bytes(B, Hq, Hkv, N, D)
+    per_split = B * Hq * (D + 2) * 4
+    assert ws % per_split == 0
+    nsplit = ws // per_split
+    assert -(-N // 4096) <= nsplit <= -(-N // 256)
+    slots = 148 * 3
+    waves = -(-(B * Hkv * -(-N // 64)) // (slots * 64))
+    assert B * Hkv * nsplit <= max(waves * slots, B * Hkv * -(-N // 4096))
